@@ -1,1 +1,170 @@
-"""B200-native DiT joint attention (placeholder; the binding is added with the C-ABI)."""
+"""B200-native DiT joint attention: Python binding of the C ABI in include/dit_attn.h.
+
+The binding only marshals arguments (tensor checks, device pointers, the
+current CUDA stream) into ``libdit_attn.so``; every step of the attention
+runs in that library's sm_100a kernel.  There is no CPU or PyTorch fallback:
+if the library is missing or cannot run, calls raise.
+
+    import attention_dit_attn_b200 as dit
+    o, lse = dit.dit_attn_fwd(q, k, v)                    # bf16 [B,H,L,D] on cuda
+    o, lse = dit.dit_attn_fwd(q8, k8, v8, q_scale=qs, k_scale=ks, v_scale=vs)  # e4m3
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+from . import _build
+
+__all__ = [
+    "DIT_ATTN_BF16", "DIT_ATTN_FP8_E4M3", "DitAttnError", "dit_attn_fwd", "dit_attn_fwd_ptr",
+    "dit_attn_status_string", "dit_attn_check_device_error", "dit_attn_set_wait_limit_ns",
+    "dit_attn_selftest_wait_timeout", "dit_attn_launches_per_call", "ensure_built", "lib",
+    "header_functions", "STATUS",
+]
+
+DIT_ATTN_BF16 = 0
+DIT_ATTN_FP8_E4M3 = 1
+
+STATUS = {
+    0: "DIT_ATTN_OK", 1: "DIT_ATTN_ERR_NULL", 2: "DIT_ATTN_ERR_SHAPE", 3: "DIT_ATTN_ERR_DTYPE",
+    4: "DIT_ATTN_ERR_ALIGN", 5: "DIT_ATTN_ERR_ARCH", 6: "DIT_ATTN_ERR_LAUNCH",
+    7: "DIT_ATTN_ERR_TIMEOUT", 8: "DIT_ATTN_ERR_VALUE",
+}
+
+HEADER = os.path.join(_build.INCLUDE, "dit_attn.h")
+
+_lib = None
+
+
+class DitAttnError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}{STATUS.get(status, status)}: {dit_attn_status_string(status)}")
+
+
+def ensure_built() -> str:
+    """Build libdit_attn.so in-tree if it is missing or older than its sources."""
+    return _build.build()
+
+
+def lib() -> ctypes.CDLL:
+    """Load the C-ABI library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_build.LIB):
+            raise RuntimeError(f"{_build.LIB} is missing: run attention_dit_attn_b200.ensure_built()")
+        L = ctypes.CDLL(_build.LIB)
+        vp, i32, u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64
+        L.dit_attn_fwd.restype = i32
+        L.dit_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, i32,
+                                   vp, vp, vp, vp]
+        L.dit_attn_status_string.restype = ctypes.c_char_p
+        L.dit_attn_status_string.argtypes = [i32]
+        L.dit_attn_check_device_error.restype = i32
+        L.dit_attn_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.dit_attn_set_wait_limit_ns.restype = None
+        L.dit_attn_set_wait_limit_ns.argtypes = [u64]
+        L.dit_attn_selftest_wait_timeout.restype = i32
+        L.dit_attn_selftest_wait_timeout.argtypes = [u64, vp]
+        L.dit_attn_launches_per_call.restype = i32
+        L.dit_attn_launches_per_call.argtypes = [i32, i32, i32, i32, i32]
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/dit_attn.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(dit_attn_\w+)\s*\(", text, flags=re.M)
+
+
+def dit_attn_status_string(status: int) -> str:
+    return lib().dit_attn_status_string(int(status)).decode()
+
+
+def _stream_handle(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def dit_attn_fwd_ptr(q: int, k: int, v: int, o: int, lse: int | None, B: int, H: int, L: int,
+                     D: int, scale: float, dtype: int, q_scale: int | None = None,
+                     k_scale: int | None = None, v_scale: int | None = None,
+                     stream: int = 0) -> int:
+    """Raw C-ABI call with integer device pointers; returns the status code."""
+    return lib().dit_attn_fwd(q, k, v, o, lse, B, H, L, D, ctypes.c_float(scale), dtype,
+                              q_scale, k_scale, v_scale, stream)
+
+
+def dit_attn_fwd(q, k, v, o=None, lse=None, *, scale: float | None = None, q_scale=None,
+                 k_scale=None, v_scale=None, want_lse: bool = True, stream=None):
+    """Attention forward on torch CUDA tensors [B, H, L, D] (bf16, or float8_e4m3fn with
+    [B, H] fp32 dequant scales).  Allocates o (bf16) and lse (fp32 [B, H, L]) when not
+    given.  Asynchronous on ``stream`` (default: torch's current stream).
+    Returns (o, lse); lse is None when want_lse is False and none was given."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [B, H, L, D] tensor")
+    if q.shape != k.shape or q.shape != v.shape or not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must share shape and dtype")
+    B, H, L, D = q.shape
+    if q.dtype == torch.bfloat16:
+        dtype = DIT_ATTN_BF16
+        scales = (None, None, None)
+        if q_scale is not None or k_scale is not None or v_scale is not None:
+            raise ValueError("scales are only for float8_e4m3fn inputs")
+    elif q.dtype == torch.float8_e4m3fn:
+        dtype = DIT_ATTN_FP8_E4M3
+        scales = []
+        for name, s in (("q_scale", q_scale), ("k_scale", k_scale), ("v_scale", v_scale)):
+            if s is None or not s.is_cuda or s.dtype != torch.float32 or s.numel() != B * H \
+                    or not s.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor with B*H elements")
+            scales.append(s.data_ptr())
+    else:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    if o is None:
+        o = torch.empty((B, H, L, D), dtype=torch.bfloat16, device=q.device)
+    elif o.shape != q.shape or o.dtype != torch.bfloat16 or not o.is_contiguous() or not o.is_cuda:
+        raise ValueError("o must be a contiguous bf16 CUDA tensor shaped like q")
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    elif lse is not None and (lse.numel() != B * H * L or lse.dtype != torch.float32
+                              or not lse.is_contiguous() or not lse.is_cuda):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor with B*H*L elements")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rc = dit_attn_fwd_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                          None if lse is None else lse.data_ptr(), B, H, L, D, float(scale), dtype,
+                          *scales, stream=_stream_handle(stream))
+    if rc != 0:
+        raise DitAttnError(rc, "dit_attn_fwd: ")
+    return o, lse
+
+
+def dit_attn_check_device_error(stream=None) -> tuple[int, int]:
+    """Synchronise, read and clear the device error word: (status, raw word)."""
+    word = ctypes.c_uint32(0)
+    rc = lib().dit_attn_check_device_error(_stream_handle(stream), ctypes.byref(word))
+    return rc, word.value
+
+
+def dit_attn_set_wait_limit_ns(ns: int) -> None:
+    lib().dit_attn_set_wait_limit_ns(int(ns))
+
+
+def dit_attn_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
+    return lib().dit_attn_selftest_wait_timeout(int(limit_ns), _stream_handle(stream))
+
+
+def dit_attn_launches_per_call(B: int, H: int, L: int, D: int, dtype: int) -> int:
+    return lib().dit_attn_launches_per_call(B, H, L, D, dtype)

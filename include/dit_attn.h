@@ -1,0 +1,127 @@
+/*
+ * dit_attn.h — C ABI of the B200 (sm_100a) DiT joint-attention forward.
+ *
+ * One call computes, for every batch entry b and head h of one DiT block,
+ * full (non-causal) multi-head joint self-attention over the concatenated
+ * text + image (or video) latent tokens:
+ *
+ *     O[b,h] = softmax(scale * Q[b,h] K[b,h]^T) V[b,h]
+ *     LSE[b,h,i] = log sum_j exp(scale * Q[b,h,i] . K[b,h,j])
+ *
+ * This is the attention core of the repeated transformer passes that
+ * dominate diffusion inference (page "How to Scale Diffusion Inference
+ * Across AMD RDNA 4 GPUs", section "Understanding the Inference Pipeline"),
+ * i.e. the operation behind the pages' selectable BF16 / FP8 attention
+ * backends (same page, section "Select an Attention Backend and Compile the
+ * Transformer"; fosswire.org summary "AMD releases xDiT configurations for
+ * scaling diffusion inference on RDNA 4 GPUs", section "Technical
+ * implementation of xDiT on RDNA 4").  The pages cite "Attention Is All You
+ * Need" and FlashAttention-2 for it (page "xDiT: an Inference Engine for
+ * Diffusion Transformers (DiTs) with Massive Parallelism", reference list);
+ * they state no formula, layout or interface, so the layout below is the
+ * plainest one ([B, H, L, D], D innermost, as in torch's SDPA).
+ *
+ * All functions are host functions, thread-safe, and never synchronise the
+ * device unless stated.  The library allocates no device memory.
+ */
+#ifndef DIT_ATTN_H
+#define DIT_ATTN_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Input element type. */
+typedef enum {
+    DIT_ATTN_BF16 = 0,      /* q, k, v bf16                                  */
+    DIT_ATTN_FP8_E4M3 = 1   /* q, k, v OCP FP8 E4M3 ("fn") + fp32 scales     */
+} dit_attn_dtype;
+
+/* Return codes. */
+typedef enum {
+    DIT_ATTN_OK = 0,
+    DIT_ATTN_ERR_NULL = 1,     /* a required pointer is NULL                 */
+    DIT_ATTN_ERR_SHAPE = 2,    /* B, H, L or D outside the supported range   */
+    DIT_ATTN_ERR_DTYPE = 3,    /* unknown dtype, or scales given for bf16    */
+    DIT_ATTN_ERR_ALIGN = 4,    /* q/k/v/o not 16-byte, lse/scales not 4-byte aligned */
+    DIT_ATTN_ERR_ARCH = 5,     /* no CUDA device, or the current device is not sm_100 */
+    DIT_ATTN_ERR_LAUNCH = 6,   /* a CUDA runtime call or the kernel launch failed */
+    DIT_ATTN_ERR_TIMEOUT = 7,  /* a device-side wait ran past its time limit */
+    DIT_ATTN_ERR_VALUE = 8     /* scale is negative, NaN or infinite         */
+} dit_attn_status;
+
+/*
+ * dit_attn_fwd — attention forward, asynchronous on `stream`.
+ *
+ * q, k, v   device pointers, contiguous [B, H, L, D] (D innermost), element
+ *           type `dtype`; 16-byte aligned.  Read only.
+ * o         device pointer, contiguous [B, H, L, D] bf16 (for both dtypes);
+ *           16-byte aligned.  Fully overwritten.
+ * lse       device pointer to [B, H, L] fp32, or NULL to skip it.  Receives
+ *           the natural-log log-sum-exp of each row's scaled logits (for
+ *           FP8, of the dequantised logits).
+ * B, H      batch entries and heads, >= 1, B*H <= 2^31-1.
+ * L         joint sequence length (text + image/video tokens), 1 <= L and
+ *           B*H*L*D < 2^40.
+ * D         head dimension: 64 or 128.
+ * scale     softmax scale, finite and >= 0 (the DiT blocks use 1/sqrt(D)).
+ * dtype     DIT_ATTN_BF16 or DIT_ATTN_FP8_E4M3.
+ * q_scale, k_scale, v_scale
+ *           FP8 only: device pointers to [B, H] fp32 per-head dequantisation
+ *           scales (x ~= s * x_hat); logits are scale*qs*ks*(q_hat.k_hat) and
+ *           O is vs * sum p v_hat / sum p.  Must be NULL for bf16.
+ * stream    CUDA stream (0 = legacy default stream).
+ *
+ * Ownership: the caller owns every buffer; the library keeps no pointer
+ * after the call returns (the kernel reads them in stream order).
+ * Errors: argument errors are reported before anything is enqueued.  A
+ * device-side wait that exceeds its limit (default 4 s) makes the kernel
+ * stop early and record an error word, reported by
+ * dit_attn_check_device_error(); the output is then undefined.
+ * Non-goals: causal masks, dropout, backward, variable-length batches.
+ */
+int dit_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                 int B, int H, int L, int D, float scale, int dtype,
+                 const float *q_scale, const float *k_scale, const float *v_scale,
+                 cudaStream_t stream);
+
+/* Static, human-readable text for a return code (never NULL). */
+const char *dit_attn_status_string(int status);
+
+/*
+ * dit_attn_check_device_error — synchronises `stream`, reads the current
+ * device's error word, clears it and returns DIT_ATTN_OK or
+ * DIT_ATTN_ERR_TIMEOUT (DIT_ATTN_ERR_LAUNCH if a CUDA call fails).  If
+ * `detail` is not NULL it receives the raw word (0 = no error; otherwise
+ * bits 0..7 the code, bits 8..15 the wait site that gave up).
+ */
+int dit_attn_check_device_error(cudaStream_t stream, uint32_t *detail);
+
+/*
+ * dit_attn_set_wait_limit_ns — time limit of every device-side wait of
+ * later launches from this process (default 4e9 ns; 0 restores it).
+ */
+void dit_attn_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * dit_attn_selftest_wait_timeout — launches one CTA whose thread waits, with
+ * the kernels' own bounded wait, on an mbarrier that nothing completes; the
+ * wait gives up after `limit_ns` and records DIT_ATTN_ERR_TIMEOUT in the
+ * error word.  Used by tests to check the timeout path without hanging the
+ * GPU.  Asynchronous on `stream`.
+ */
+int dit_attn_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+
+/*
+ * dit_attn_launches_per_call — number of kernel launches one dit_attn_fwd
+ * call with these arguments enqueues (for launch accounting).
+ */
+int dit_attn_launches_per_call(int B, int H, int L, int D, int dtype);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DIT_ATTN_H */

@@ -1,0 +1,71 @@
+"""Host-side checks of the C ABI library (no GPU needed, no kernel launched)."""
+import ctypes
+import re
+
+import pytest
+import torch
+
+import attention_dit_attn_b200 as dit
+
+
+@pytest.fixture(scope="module")
+def L():
+    dit.ensure_built()
+    return dit.lib()
+
+
+def test_library_exports_every_header_function(L):
+    names = dit.header_functions()
+    assert set(names) == {"dit_attn_fwd", "dit_attn_status_string", "dit_attn_check_device_error",
+                          "dit_attn_set_wait_limit_ns", "dit_attn_selftest_wait_timeout",
+                          "dit_attn_launches_per_call"}
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_header_status_codes_match_binding():
+    text = open(dit.HEADER).read()
+    codes = dict((name, int(val)) for name, val in re.findall(r"(DIT_ATTN_(?:OK|ERR_\w+))\s*=\s*(\d+)", text))
+    assert {v: k for k, v in codes.items()} == dit.STATUS
+
+
+def test_status_strings(L):
+    for code in dit.STATUS:
+        s = dit.dit_attn_status_string(code)
+        assert s and s != "unknown status"
+    assert dit.dit_attn_status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("args,want", [
+    ((0, 16, 16, 16, None, 1, 1, 8, 64, 0.1, 0), 1),             # q NULL
+    ((16, 16, 16, 0, None, 1, 1, 8, 64, 0.1, 0), 1),             # o NULL
+    ((16, 16, 16, 16, None, 1, 1, 8, 64, 0.1, 5), 3),            # bad dtype
+    ((16, 16, 16, 16, None, 1, 1, 8, 64, 0.1, 1), 1),            # fp8 without scales
+    ((16, 16, 16, 16, None, 1, 1, 8, 64, 0.1, 0, 16), 3),        # bf16 with a scale
+    ((16, 16, 16, 16, None, 0, 1, 8, 64, 0.1, 0), 2),            # B = 0
+    ((16, 16, 16, 16, None, 1, 1, 0, 64, 0.1, 0), 2),            # L = 0
+    ((16, 16, 16, 16, None, 1, 1, 8, 80, 0.1, 0), 2),            # D = 80
+    ((16, 16, 16, 16, None, 1 << 20, 1 << 11, 1 << 10, 128, 0.1, 0), 2),  # > 2^40 elements
+    ((24, 16, 16, 16, None, 1, 1, 8, 64, 0.1, 0), 4),            # q misaligned
+    ((16, 16, 16, 16, 18, 1, 1, 8, 64, 0.1, 0), 4),              # lse misaligned
+    ((16, 16, 16, 16, None, 1, 1, 8, 64, float("nan"), 0), 8),   # scale NaN
+    ((16, 16, 16, 16, None, 1, 1, 8, 64, -0.5, 0), 8),           # scale < 0
+])
+def test_argument_validation_before_any_cuda_call(L, args, want):
+    assert dit.dit_attn_fwd_ptr(*args) == want
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a GPU")
+def test_wellformed_call_without_gpu_reports_arch(L):
+    assert dit.dit_attn_fwd_ptr(16, 16, 16, 16, None, 1, 1, 8, 64, 0.1, 0) == 5
+    assert L.dit_attn_selftest_wait_timeout(1000, None) == 5
+
+
+def test_launch_accounting(L):
+    assert dit.dit_attn_launches_per_call(2, 24, 16896, 128, 0) == 1
+
+
+def test_python_binding_rejects_cpu_tensors():
+    x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        dit.dit_attn_fwd(x, x, x)
