@@ -75,6 +75,14 @@ WORKLOADS = {
 # Same five, in the order the workload list gives them.
 ORDER = ["tiny_256", "flux_1024x768", "flux_2048_cfg", "sd35_1024_fp8", "wan_720p_81f"]
 
+# Profiling-size slices of the workloads above (same L and D, fewer heads): inputs
+# still larger than the 126 MB L2, small enough for a multi-pass ncu capture.
+PROFILE_CASES = {
+    "flux_2048_h16": Workload("flux_2048_h16", B=1, H=16, L=512 + 16384, D=128, dtype="bf16",
+                              seed=1003, text_rows=512, text_scale=2.0),
+}
+ALL = {**WORKLOADS, **PROFILE_CASES}
+
 
 @dataclass
 class Inputs:

@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Bench of the DiT joint-attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one dit_attn_fwd call over one batch of synthetic inputs (the whole
+hot path is one kernel launch).  Prints ONE JSON line on rank 0.
+
+* value: attention TFLOP/s (4*B*H*L^2*D per call) over all ranks, inputs
+  resident in HBM, timed with CUDA events between barriers; max over ranks.
+* e2e: the same metric through the public API with the step's q/k/v copied
+  from pinned host memory and o/lse copied back, inside the timed region.
+* roofline: the attention kernel against the measured bf16 (or derived fp8)
+  tensor peak.
+* cpu_baseline: the fp64 oracle on this host's cores over a bounded sample of
+  the workload's query rows (rank 0, N=1 only).
+* --impl reference: the oracle alone, as the reference arm, on the same
+  workload and metric.
+Multi-GPU (torchrun): every rank runs its own replica (no data exchange:
+heads and batches are independent), scaling "weak".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOP/s and % of B200 tensor-core peak at 1 GPU"
+DEFAULT_WORKLOAD = "flux_2048_cfg"      # the first workload with L >= 16k (the stated target)
+NOMINAL_TFLOPS = {"bf16": 2250.0, "e4m3": 4500.0}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ------------------------------------------------------------------ small helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "attention_dit_attn_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (its source hash matches); else None."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self):
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self, gpu_index: int | None):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                idx = int(parts[0])
+                if gpu_index is not None and idx != gpu_index:
+                    continue
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def physical_gpu_index(local_rank: int):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+        return None
+    return local_rank
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+class Dist:
+    def __init__(self, n_gpus: int, backend: str | None = None):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend=backend or "nccl",
+                                    timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+        if n_gpus != self.world and self.world > 1:
+            print(f"warning: --gpus {n_gpus} but WORLD_SIZE {self.world}", file=sys.stderr)
+
+    @classmethod
+    def single(cls):
+        d = cls.__new__(cls)
+        d.world, d.rank, d.local_rank, d.pg = 1, 0, 0, None
+        return d
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float, device=None) -> float:
+        if self.pg is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def aggregate(per_rank_flops: float, steps: int, world: int, max_seconds: float) -> float:
+    """Whole-job TFLOP/s: the work of every rank over the slowest rank's time."""
+    return per_rank_flops * steps * world / max_seconds / 1e12
+
+
+# ------------------------------------------------------------------ CPU (oracle) timing
+
+def oracle_sample_time(w, inp, n_rows: int, n_heads: int = 1, nthreads: int = 0):
+    """Time the fp64 oracle on n_rows sampled query rows of each of the first n_heads
+    heads of batch entry 0 (all L keys each); returns (seconds, flops)."""
+    import oracle
+    from attention_dit_attn_b200 import workloads as wl
+    n_heads = max(1, min(n_heads, w.H))
+    q = wl.as_bits(inp.q[:1, :n_heads])
+    k = wl.as_bits(inp.k[:1, :n_heads])
+    v = wl.as_bits(inp.v[:1, :n_heads])
+    rows = wl.sample_rows(1, n_heads, w.L, min(n_rows, w.L), w.seed)
+    kw = {}
+    dtype = oracle.BF16
+    if inp.q_scale is not None:
+        dtype = oracle.E4M3
+        kw = dict(q_scale=inp.q_scale[:1, :n_heads].numpy(), k_scale=inp.k_scale[:1, :n_heads].numpy(),
+                  v_scale=inp.v_scale[:1, :n_heads].numpy())
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, w.scale, dtype=dtype, rows=rows, nthreads=nthreads, **kw)
+    dt = time.perf_counter() - t0
+    return dt, 4.0 * w.L * w.D * rows.size
+
+
+def plan_sample(w, inp, seconds: float):
+    """(rows per head, heads) so that the oracle runs for about `seconds`."""
+    probe = min(w.L, 256)
+    dt, _ = oracle_sample_time(w, inp, probe)
+    per_row = max(dt / probe, 1e-7)
+    total = max(16, int(seconds / per_row))
+    if total <= w.L:
+        return total, 1
+    heads = min(w.H, -(-total // w.L))
+    return w.L, heads
+
+
+def cpu_baseline(w, inp, seconds: float = 15.0):
+    import oracle
+    rows, heads = plan_sample(w, inp, seconds)
+    dt, flops = oracle_sample_time(w, inp, rows, heads)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 oracle on {rows} sampled query rows x {heads} head(s) of batch 0 of "
+                      f"{w.name} (all {w.L} keys per row): {dt:.1f} s on {oracle.max_threads()} threads"}
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args, dist: Dist):
+    """Reference arm: the fp64 CPU oracle as it stands (no GPU)."""
+    if dist.rank != 0:
+        return
+    import oracle
+    from attention_dit_attn_b200 import workloads as wl
+    w = wl.ALL[args.workload]
+    inp = wl.generate_workload(w)
+    total_budget = 120.0
+    rows, heads = plan_sample(w, inp, total_budget / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample_time(w, inp, rows, heads)
+    t_total, f_total = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample_time(w, inp, rows, heads)
+        t_total += dt
+        f_total += fl
+    value = f_total / t_total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: fp64 oracle on {rows} sampled query rows x {heads} "
+                                   f"head(s) of batch 0 of {w.name} (all {w.L} keys per row)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    in_bytes = 3 * w.B * w.H * w.L * w.D * (1 if w.dtype == "e4m3" else 2)
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "D": w.D, "text_tokens": w.text_rows,
+            "input_dtype": w.dtype, "output_dtype": "bf16", "causal": False,
+            "inputs_bytes": in_bytes,
+            "l2": ("inputs larger than L2 (%.0f MB > 126 MB)" % (in_bytes / 1e6)) if in_bytes > L2_BYTES
+            else "L2 flushed between timed steps (256 MB write)",
+            "parallelism": "replicas"}
+
+
+def run_ours(args, dist: Dist):
+    import torch
+    import attention_dit_attn_b200 as dit
+    from attention_dit_attn_b200 import workloads as wl
+
+    dit.ensure_built()
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    w = wl.ALL[args.workload]
+    inp = wl.generate_workload(w)
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    kw = {}
+    if inp.q_scale is not None:
+        kw = dict(q_scale=inp.q_scale.to(dev).contiguous(), k_scale=inp.k_scale.to(dev).contiguous(),
+                  v_scale=inp.v_scale.to(dev).contiguous())
+    o = torch.empty((w.B, w.H, w.L, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    cfg = workload_config(w)
+    flush = None
+    if cfg["inputs_bytes"] <= L2_BYTES:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if flush is not None:
+            flush.fill_(1)
+        dit.dit_attn_fwd(q, k, v, o, lse, scale=w.scale, stream=stream, **kw)
+
+    # ---- device-resident timing
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    rc, word = dit.dit_attn_check_device_error(stream)
+    if rc != 0:
+        raise RuntimeError(f"device error during warm-up: {word:#x}")
+    sampler = ClockSampler()
+    if dist.rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if flush is None:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        kernel_ms_total = e0.elapsed_time(e1)
+        seconds = kernel_ms_total / 1e3
+    else:
+        # Flush between steps; time only the attention launches (per-launch events).
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        e0.record(stream)
+        for a, b in evs:
+            flush.fill_(1)
+            a.record(stream)
+            dit.dit_attn_fwd(q, k, v, o, lse, scale=w.scale, stream=stream, **kw)
+            b.record(stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        kernel_ms_total = sum(a.elapsed_time(b) for a, b in evs)
+        seconds = kernel_ms_total / 1e3
+    dist.barrier()
+    if dist.rank == 0:
+        time.sleep(0.2)
+        sampler.stop()
+    rc, word = dit.dit_attn_check_device_error(stream)
+    if rc != 0:
+        raise RuntimeError(f"device error during the timed region: {word:#x}")
+    max_seconds = dist.max(seconds, dev)
+    value = aggregate(w.flops, args.steps, dist.world, max_seconds)
+    kernel_avg_s = kernel_ms_total / 1e3 / args.steps
+    launches = args.steps * dit.dit_attn_launches_per_call(w.B, w.H, w.L, w.D, 0 if w.dtype == "bf16" else 1)
+
+    # ---- end to end through the public API, host buffers, copies in the timed region
+    e2e_steps = max(3, min(args.steps, 10))
+    hq, hk, hv = (t.pin_memory() for t in (inp.q, inp.k, inp.v))
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dit.dit_attn_fwd(dq, dk, dv, o, lse, scale=w.scale, stream=stream, **kw)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = dist.max(a.elapsed_time(b) / 1e3, dev)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    e2e_ok = torch.equal(ho, o.cpu())
+
+    peaks, peaks_kind = load_peaks()
+    if w.dtype == "bf16":
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        peak_note = f"bf16 dense, {peaks_kind} (burst)"
+    else:
+        # FP8 contraction: measured bf16 peak x the nominal fp8/bf16 ratio (2x).
+        peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        peak_note = f"fp8 dense = 2 x bf16 {peaks_kind} (burst)"
+    achieved = w.flops / kernel_avg_s / 1e12
+    traffic = profiled_traffic(w.name)
+    clocks = sampler.summary(physical_gpu_index(dist.local_rank)) if dist.rank == 0 else {}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * max_seconds / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic",
+        "config": cfg,
+        "pct_of_peak": {"nominal_dense": 100.0 * value / dist.world / NOMINAL_TFLOPS[w.dtype],
+                        "nominal_tflops": NOMINAL_TFLOPS[w.dtype]},
+        "e2e": {"value": aggregate(w.flops, e2e_steps, dist.world, e2e_s), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "result_matches_device": e2e_ok},
+        "gpu_launches": launches,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_source": peak_note, "traffic": traffic,
+                     "kernel": "dit::attn_fwd_kernel", "flops_per_launch": w.flops},
+        "clocks": clocks,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from attention_dit_attn_b200 import workloads as wl
+    if args.workload not in wl.ALL:
+        ap.error(f"--workload must be one of {list(wl.ALL)}")
+    if args.impl == "reference":
+        # The oracle runs on rank 0's host cores only; other ranks exit at once.
+        if int(os.environ.get("RANK", "0")) == 0:
+            run_reference(args, Dist.single())
+        return
+    dist = Dist(args.gpus)
+    try:
+        run_ours(args, dist)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()
