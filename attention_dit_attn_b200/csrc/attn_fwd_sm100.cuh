@@ -121,6 +121,11 @@ struct KCfg {
     // different register budgets does not allocate.
     static constexpr int THREADS = 384;
     static constexpr int REGS_SOFTMAX = 208, REGS_OTHER = 88;
+    // Element pairs (of every 8) whose exponential runs on the FMA pipe.
+#ifndef DIT_EXP_EMU
+#define DIT_EXP_EMU 2
+#endif
+    static constexpr int EXP_EMU = DIT_EXP_EMU;
     static_assert(2 * REGS_SOFTMAX + REGS_OTHER == 3 * 168, "register split = launch budget");
     // Instruction descriptors (M = 128 rows).
     static constexpr uint32_t IDESC_QK =
@@ -230,11 +235,44 @@ __device__ __forceinline__ uint32_t swz(uint32_t off)
 
 // ------------------------------------------------------------------ softmax of one S tile
 
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^x for a pair, on the FMA/ALU pipes instead of MUFU.  x = n + f with
+// n = rint(x) (adding 1.5*2^23 leaves rint(x) in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f is a cubic fitted for minimum max relative error on
+// [-1/2, 1/2] (max rel. error 7.5e-5, below the half-ulp of bf16 and f16 P);
+// 2^n is added to the exponent field.  x is clamped to >= -126 so the
+// exponent never underflows; the callers guarantee x <= 9.
+constexpr float kPolyC0 = 0.9999281167984009f, kPolyC1 = 0.6932609677314758f,
+                kPolyC2 = 0.24261052906513214f, kPolyC3 = 0.05517127364873886f;
+constexpr float kRintMagic = 12582912.0f;   // 1.5 * 2^23
+
+__device__ __forceinline__ float2 exp2_poly2(float2 x)
+{
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    const float2 t = __fadd2_rn(x, make_float2(kRintMagic, kRintMagic));
+    const float2 n = __fadd2_rn(t, make_float2(-kRintMagic, -kRintMagic));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+    float2 q = __ffma2_rn(f, make_float2(kPolyC3, kPolyC3), make_float2(kPolyC2, kPolyC2));
+    q = __ffma2_rn(q, f, make_float2(kPolyC1, kPolyC1));
+    q = __ffma2_rn(q, f, make_float2(kPolyC0, kPolyC0));
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Loads this thread's row of S (128 fp32), updates the running max / sum,
-// rescales O when needed, and writes P (16-bit) over the S columns.  P chunk
+// writes P (16-bit) over the S columns and rescales O when needed.  P chunk
 // i (S columns 32i..32i+31) goes to columns 16i..16i+15, which hold S values
-// already consumed, so P can be stored chunk by chunk.
-template <class C, bool MASK>
+// already consumed, so P can be stored chunk by chunk.  Of every 8 element
+// pairs, EMU pairs take 2^x from exp2_poly2 (FMA pipe), the rest from MUFU,
+// which balances the two pipes.
+template <class C, bool MASK, int EMU>
 __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int valid, bool first,
                                              float c2, float &m_use, float &l)
 {
@@ -244,17 +282,26 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int valid
         tmem_ld32(tS + 32 * i, s[i]);
     tmem_wait_ld();
 
-    float mx0 = -INFINITY, mx1 = -INFINITY;
+    if (MASK) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-            if (!MASK || 32 * i + c < valid)
-                mx0 = fmaxf(mx0, __uint_as_float(s[i][c]));
-            if (!MASK || 32 * i + c + 1 < valid)
-                mx1 = fmaxf(mx1, __uint_as_float(s[i][c + 1]));
-        }
-    const float mx = fmaxf(mx0, mx1);
+            for (int c = 0; c < 32; ++c)
+                if (32 * i + c >= valid)
+                    s[i][c] = __float_as_uint(-INFINITY);
+    }
+    // Row max: 8 independent chains of 3-input max, then a short tree.
+    float m8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        m8[k] = fmaxf(__uint_as_float(s[0][2 * k]), __uint_as_float(s[0][2 * k + 1]));
+#pragma unroll
+    for (int e = 16; e < 128; e += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            m8[k] = max3f(m8[k], __uint_as_float(s[e >> 5][(e & 31) + 2 * k]),
+                          __uint_as_float(s[e >> 5][(e & 31) + 2 * k + 1]));
+    const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
 
     float alpha = 1.f;
     if (first) {
@@ -264,27 +311,40 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int valid
         m_use = mx;
     }
     const float mc = m_use * c2;
+    const float2 c2c2 = make_float2(c2, c2), nmc = make_float2(-mc, -mc);
 
-    float sum0 = 0.f, sum1 = 0.f;
+    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                     make_float2(0.f, 0.f)};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-            float a = ex2_approx(fmaf(__uint_as_float(s[i][c]), c2, -mc));
-            float b = ex2_approx(fmaf(__uint_as_float(s[i][c + 1]), c2, -mc));
-            if (MASK) {
-                a = (32 * i + c < valid) ? a : 0.f;
-                b = (32 * i + c + 1 < valid) ? b : 0.f;
+            const int pi = (32 * i + c) >> 1;     // pair index 0..63
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[i][c]), __uint_as_float(s[i][c + 1])),
+                                        c2c2, nmc);
+            float2 e;
+            if ((pi & 7) >= 8 - EMU) {
+                e = exp2_poly2(x);
+            } else {
+                e.x = ex2_approx(x.x);
+                e.y = ex2_approx(x.y);
             }
-            sum0 += a;
-            sum1 += b;
-            pk[c / 2] = pack_p(a, b, C::FP8);
+            if (MASK) {
+                e.x = (32 * i + c < valid) ? e.x : 0.f;
+                e.y = (32 * i + c + 1 < valid) ? e.y : 0.f;
+            }
+            acc[pi & 3] = __fadd2_rn(acc[pi & 3], e);
+            pk[c / 2] = pack_p(e.x, e.y, C::FP8);
         }
         tmem_st16(tS + 16 * i, pk);
     }
-    l = l * alpha + (sum0 + sum1);
-    // After the exponentials (S registers dead).  O is stable here (S_g(j) complete implies PV_g(j-1) complete).
+    const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+    const float2 a = __fadd2_rn(a01, a23);
+    l = l * alpha + (a.x + a.y);
+
+    // After the exponentials (S registers dead).  O is stable here: S_g(j)
+    // complete implies PV_g(j-1) complete.
     if (!first && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int cc = 0; cc < C::D / 32; ++cc) {
@@ -297,7 +357,6 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int valid
             tmem_st32(tO + 32 * cc, o);
         }
     }
-
     tmem_wait_st();
 }
 
@@ -544,9 +603,9 @@ __device__ __forceinline__ void softmax_role(const Ctx<C> &x, const FwdParams &p
         }
         tc_fence_after();
         if (j + 1 < p.n_kv || p.kv_tail == kBN)
-            softmax_tile<C, false>(tS, tO, kBN, j == 0, c2, m_use, l);
+            softmax_tile<C, false, C::EXP_EMU>(tS, tO, kBN, j == 0, c2, m_use, l);
         else
-            softmax_tile<C, true>(tS, tO, p.kv_tail, j == 0, c2, m_use, l);
+            softmax_tile<C, true, C::EXP_EMU>(tS, tO, p.kv_tail, j == 0, c2, m_use, l);
         tc_fence_before();
         mbar_arrive(x.bar(bars->p_full[g]));
     }
