@@ -1,165 +1,139 @@
-// Flash-style attention forward for B200 (sm_100a): TMA-staged Q/K/V tiles,
-// tcgen05 MMAs with TMEM accumulators, online fp32 softmax, warp-specialised
-// roles, bf16 and FP8-E4M3 inputs.
+// Attention forward on a CTA pair (cluster of 2, tcgen05 cta_group::2).
 //
-// Operation: O = softmax(scale * Q K^T) V per (batch, head) with the fp32
-// log-sum-exp of each row, the attention core of a DiT block (page "How to
-// Scale Diffusion Inference Across AMD RDNA 4 GPUs", sections "Understanding
-// the Inference Pipeline" and "Select an Attention Backend and Compile the
-// Transformer").  The tiling with a running max and running sum is the
-// FlashAttention-2 scheme the pages cite (page "xDiT: an Inference Engine for
-// Diffusion Transformers (DiTs) with Massive Parallelism", reference list),
-// re-designed here for tcgen05 / TMEM.
+// O = softmax(scale * Q K^T) V plus the row log-sum-exp (operation and
+// sources: attn_common.cuh).  A cluster of two CTAs on two SMs processes 256 query
+// rows of one (b, h); each CTA owns 128 of them.  Every MMA is issued once,
+// by the leader CTA, with M = 256:
 //
-// One CTA owns a pair of 128-row query tiles of one (b, h) and streams all
-// K/V tiles of that head through a shared-memory ring:
+//   S = Q K^T   A = each CTA's own Q tile, B = K tile split by keys: each CTA
+//               loads 64 of the tile's 128 keys;
+//   O += P V    A = P from each CTA's TMEM, B = V tile split by columns: each
+//               CTA loads D/2 of the D columns.
 //
-//   warps 0-3   softmax + epilogue of query tile 0 (one thread per row)
-//   warps 4-7   softmax + epilogue of query tile 1
-//   warp  8     TMA producer (Q once, then K_j, V_j into the ring)
-//   warp  9     MMA issuer (one thread) and TMEM owner
-//   warps 10-11 FP8 only: convert each e4m3 V tile to f16 in shared memory
+// So each SM streams only half of every K/V tile from L2 while the MMA sees
+// the full tile, without TMA multicast.
 //
-// TMEM (512 columns x 128 lanes of 32 bit): S0 | S1 | O0 | O1.  S_g holds the
-// fp32 logits of tile g; the softmax overwrites its first 64 (bf16/f16 P)
-// columns with P, which the PV MMA reads straight from TMEM.  MMA issue order
-//   S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
-// lets one tile's softmax overlap the other tile's MMAs (ping-pong).  The
-// MMAs of one thread run in issue order, so S_g(j+1) (which overwrites P_g(j))
-// starts after PV_g(j), and when S_g(j+1) is complete O_g is stable, which is
-// when the softmax rescales it.
+// Split keys: each query row is handled by two threads (warps w and w+4 share
+// TMEM lanes 32(w%4)..+31).  Half h owns keys 64h..64h+63 of every K/V tile
+// and keeps its own running max, running sum and output accumulator O_h
+// (a flash-style split over keys); the two partial results are merged once,
+// in the epilogue, through their log-sum-exp.  No per-tile exchange between
+// the two threads is needed.  TMEM (per CTA, 512 columns): two S buffers of
+// 128 columns, O_0 and O_1 of D columns each.  The MMA issues S(j+2) right
+// after PV(j) into the same buffer, so the softmax of step j+1 overlaps
+// PV(j) and S(j+2).
 //
-// Rescaling is lazy: a row keeps its running max m while the new tile's max
-// exceeds it by at most kRescaleLog2 (in log2 units), so p <= 2^kRescaleLog2;
-// O and l are only rescaled when the max grows further.  The result is exact
-// because O and l always share the same max.
+// Warps (per CTA):
+//   0-3, 4-7  softmax + epilogue (half h = warp / 4)
+//   8         TMA producers (lane 0: Q and K, lane 1: V; both CTAs load halves)
+//   9         TMEM owner; in the leader also the single MMA-issuing thread
+//   10-11     FP8 only: e4m3 -> f16 conversion of this CTA's V half
 //
-// Every wait is bounded by a time limit; on expiry the kernel records an
-// error word, the roles drain their in-flight copies/MMAs and the CTA exits.
+// P of half h is written over S columns 64h..64h+31 of its buffer (values
+// only that thread has read), and the PV MMA reads it from there.  O_h is
+// rescaled lazily: a rescale at step j first waits for PV(j-1); per-buffer
+// barriers keep every parity wait unambiguous (S(j) complete implies PV(j-2)
+// complete, and S(j+2) / PV(j+2) cannot complete before this step's P).
 #pragma once
-#include <cuda_bf16.h>
-#include <cuda_fp16.h>
-
-#include "sm100_ptx.cuh"
+#include "attn_common.cuh"
 
 namespace dit {
 
-constexpr int kBM = 128;             // query rows per tile (MMA M)
-constexpr int kBN = 128;             // keys per K/V tile
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleLog2 = 8.0f; // lazy-rescale threshold (p <= 256)
-
-// Wait sites recorded in the error word (bits 8..15).
-enum : uint32_t {
-    kSiteQFull = 1, kSiteKFull = 2, kSitePFull = 3, kSiteVhFull = 4, kSiteKvEmpty = 5,
-    kSiteSFull = 6, kSiteOFull = 7, kSiteConvFull = 8, kSiteVhEmpty = 9, kSiteDrain = 10,
-    kSiteSelftest = 11
-};
-constexpr uint32_t kErrTimeout = 7;  // same value as DIT_ATTN_ERR_TIMEOUT
-
-__device__ unsigned int g_error_word;
-
-struct FwdParams {
-    int L;
-    int n_kv;          // ceil(L / kBN)
-    int n_pairs;       // ceil(ceil(L / kBM) / 2)
-    int kv_tail;       // valid keys in the last K/V tile, 1..128
-    float scale;       // softmax scale
-    const float *q_scale;  // FP8: [B*H] dequant scales
-    const float *k_scale;
-    const float *v_scale;
-    float *lse;        // [B*H*L] or null
-    unsigned long long wait_limit_ns;
-};
-
-__host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
+#ifndef DIT_PAIR_EXP_EMU
+#define DIT_PAIR_EXP_EMU 2
+#endif
 
 template <int D_, bool FP8_>
-struct KCfg {
+struct PCfg {
     static constexpr int D = D_;
     static constexpr bool FP8 = FP8_;
-    static constexpr int ELT = FP8 ? 1 : 2;              // bytes per input element
-    static constexpr int ROW = D * ELT;                  // bytes per Q/K/V row
-    static constexpr int SWZ = ROW >= 128 ? 128 : 64;    // swizzle span of Q/K/V tiles
+    static constexpr int ELT = FP8 ? 1 : 2;
+    static constexpr int ROW = D * ELT;                    // Q/K row bytes
+    static constexpr int SWZ = ROW >= 128 ? 128 : 64;      // Q/K swizzle span
     static constexpr uint32_t SWZ_MODE = SWZ == 128 ? kSwizzle128B : kSwizzle64B;
-    static constexpr int BOX_ELEMS = SWZ / ELT;          // elements per TMA box row
-    static constexpr int NBOX = D / BOX_ELEMS;           // TMA boxes per tile
-    static constexpr int BOX_BYTES = kBM * SWZ;
-    static constexpr int TILE = kBM * ROW;               // one Q/K/V tile in smem
-    static constexpr int KSTEP = 32;                     // bytes of K per MMA: 16 x 16-bit or 32 x 8-bit
+    static constexpr int BOX_ELEMS = SWZ / ELT;
+    static constexpr int NBOX = ROW / SWZ;
+    static constexpr int QBOX_BYTES = kBM * SWZ;
+    static constexpr int QTILE = kBM * ROW;
+    static constexpr int KROWS = kBN / 2;                  // keys per CTA per tile
+    static constexpr int KBOX_BYTES = KROWS * SWZ;
+    static constexpr int KTILE = KROWS * ROW;
+    static constexpr int KSTEP = 32;
     static constexpr int QK_STEPS = ROW / KSTEP;
     static constexpr int STEPS_PER_BOX = SWZ / KSTEP;
-    // 16-bit V operand of the PV MMA (bf16 or f16), MN-major, 128B swizzle.
-    static constexpr int VROW = D * 2;
-    static constexpr int VBOX_BYTES = kBN * 128;
-    static constexpr int VTILE = kBN * VROW;
-    static constexpr int PV_STEPS = kBN / 16;
-    // 16-bit O staging tile for the TMA store, 128B swizzle, 64 columns per box.
-    static constexpr int OBOX = (D * 2) / 128;
-    static constexpr int OBOX_BYTES = kBM * 128;
-    static constexpr int OTILE = kBM * D * 2;
-    static constexpr int NSTAGE = FP8 ? (D == 64 ? 8 : 4) : (D == 64 ? 8 : 4);
-    // Shared-memory layout (offsets from a 1024-byte aligned base).
+    // V half as loaded: 128 keys x D/2 elements (row = swizzle span).
+    static constexpr int VRAW_ROW = (D / 2) * ELT;
+    static constexpr int VRAW_TILE = kBN * VRAW_ROW;
+    // 16-bit V operand of PV: 128 keys x D/2, MN-major, row = swizzle span.
+    static constexpr int VROW = D;
+    static constexpr uint32_t V_SWZ_MODE = VROW == 128 ? kSwizzle128B : kSwizzle64B;
+    static constexpr int VTILE16 = kBN * VROW;
+    static constexpr int NK = 2, NV = 2, NVH = 2;   // K(j), V(j) live in stage j % 2
+    // O staging (bf16, 128 rows, SW128 boxes of 64 columns).
+    static constexpr int OBOX = (D * 2) / 128, OBOX_BYTES = kBM * 128, OTILE = kBM * D * 2;
+    // Shared memory (offsets from a 1024-aligned base).
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_KV = OFF_Q + 2 * align_up(TILE, 1024);
-    static constexpr int OFF_VH = OFF_KV + NSTAGE * align_up(TILE, 1024);
-    static constexpr int OFF_OST = OFF_VH + (FP8 ? 2 * VTILE : 0);
-    static constexpr int OFF_BAR = OFF_OST + (FP8 ? 2 * OTILE : 0);
-    static constexpr int BAR_BYTES = 256;
-    static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
+    static constexpr int OFF_K = OFF_Q + align_up(QTILE, 1024);
+    static constexpr int OFF_V = OFF_K + NK * align_up(KTILE, 1024);
+    static constexpr int OFF_VH = OFF_V + NV * align_up(VRAW_TILE, 1024);
+    static constexpr int OFF_OST = OFF_VH + (FP8 ? NVH * align_up(VTILE16, 1024) : 0);
+    static constexpr int OFF_RED = OFF_OST + (FP8 ? OTILE : 0);
+    static constexpr int RED_BYTES = 2 * 2 * kBM * 4;      // [m|l][half][row] floats (epilogue merge)
+    static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
+    static constexpr int BAR_BYTES = 512;
+    // At least 116 KB so two CTAs never share an SM (each holds all 512 TMEM columns).
+    static constexpr int SMEM_RAW = OFF_BAR + BAR_BYTES + 1024;
+    static constexpr int SMEM_BYTES = SMEM_RAW > 118784 ? SMEM_RAW : 118784;
     // TMEM columns.
-    static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
+    static constexpr uint32_t TM_S = 0;                    // buffer b at 128 b (b = 0, 1)
+    static constexpr uint32_t TM_O = 256;                  // O_h at TM_O + h * D
     static constexpr uint32_t TMEM_COLS = 512;
-    // Warp roles.
-    static constexpr int TMA_WARP = 8, MMA_WARP = 9, CONV_WARP0 = 10;
-    static constexpr int CONV_THREADS = FP8 ? 64 : 0;
-    // Three full warpgroups for every variant, so setmaxnreg can move registers
-    // from warpgroup 2 (TMA, MMA, converter) to the two softmax warpgroups:
-    // 12 warps x 168 launch registers = (2 x 208 + 88) x 128 threads.  The
-    // wait helpers are all inlined: a real call across warpgroups with
-    // different register budgets does not allocate.
+    // Warp roles / registers.
+    static constexpr int TMA_WARP = 8, MMA_WARP = 9, CONV_WARP0 = 10, CONV_THREADS = 64;
     static constexpr int THREADS = 384;
-    static constexpr int REGS_SOFTMAX = 208, REGS_OTHER = 88;
-    // Element pairs (of every 8) whose exponential runs on the FMA pipe.
-#ifndef DIT_EXP_EMU
-#define DIT_EXP_EMU 2
-#endif
-    static constexpr int EXP_EMU = DIT_EXP_EMU;
-    static_assert(2 * REGS_SOFTMAX + REGS_OTHER == 3 * 168, "register split = launch budget");
-    // Instruction descriptors (M = 128 rows).
-    static constexpr uint32_t IDESC_QK =
-        FP8 ? make_idesc(kFmtE4M3, kFmtE4M3, 0, kBM, kBN) : make_idesc(kFmtBF16, kFmtBF16, 0, kBM, kBN);
-    static constexpr uint32_t IDESC_PV =
-        FP8 ? make_idesc(kFmtF16, kFmtF16, 1, kBM, D) : make_idesc(kFmtBF16, kFmtBF16, 1, kBM, D);
+    static constexpr int REGS_SOFTMAX = 224, REGS_OTHER = 56;   // 2 x 224 + 56 = 3 x 168
+    static constexpr int EXP_EMU = DIT_PAIR_EXP_EMU;
+    static constexpr uint32_t IDESC_QK = FP8 ? make_idesc(kFmtE4M3, kFmtE4M3, 0, 2 * kBM, kBN)
+                                             : make_idesc(kFmtBF16, kFmtBF16, 0, 2 * kBM, kBN);
+    static constexpr uint32_t IDESC_PV = FP8 ? make_idesc(kFmtF16, kFmtF16, 1, 2 * kBM, D)
+                                             : make_idesc(kFmtBF16, kFmtBF16, 1, 2 * kBM, D);
 
     static_assert(D == 64 || D == 128, "head dim");
-    static_assert(NBOX * BOX_BYTES == TILE, "tile = whole boxes");
+    static_assert(NBOX * QBOX_BYTES == QTILE && NBOX * KBOX_BYTES == KTILE, "whole boxes");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    static_assert(TM_O1 + D <= TMEM_COLS, "TMEM budget");
+    static_assert(TM_O + 2 * D <= TMEM_COLS, "TMEM budget");
 };
 
-// Barrier block in shared memory.
-template <int NS>
-struct Bars {
-    uint64_t q_full;
-    uint64_t kv_full[NS];
-    uint64_t kv_empty[NS];
-    uint64_t s_full[2];
-    uint64_t p_full[2];
-    uint64_t o_full[2];
-    uint64_t vh_full[2];
-    uint64_t vh_empty[2];
+struct PairBars {
+    uint64_t q_full;          // leader: both CTAs' Q tiles landed
+    uint64_t k0_full;         // leader: K(0..1), both halves, landed
+    uint64_t ready[2];        // leader: everything step j needs (b = j % 2): P(j) from
+                              // the 16 softmax warps, V(j), K(j+2)
+    uint64_t v_full[2];       // fp8: this CTA's raw V(j) half landed (converter input)
+    uint64_t s_full[2];       // each CTA: S buffer b holds S(j); frees K stage b
+    uint64_t pv_done[2];      // each CTA: PV(j) complete; frees V stage b
     uint64_t drain;
     uint32_t tmem_base;
     uint32_t abort;
 };
 
-// ------------------------------------------------------------------ bounded waits
+template <class C>
+struct PairCtx {
+    PairBars *bars;
+    uint8_t *sm;              // generic pointer to the aligned shared-memory base
+    uint32_t base, tmem, rank;
+    volatile uint32_t *abort;
+    unsigned long long lim;
+    int bh, q0;               // q0: first query row of this CTA's tile
+    __device__ uint32_t bar(const uint64_t &b) const { return smem_u32(&b); }
+    __device__ uint32_t leader_bar(const uint64_t &b) const { return mapa_shared(smem_u32(&b), 0); }
+};
 
-__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t *abort,
-                                       unsigned long long limit, uint32_t site)
+__device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, volatile uint32_t *abort,
+                                                 unsigned long long limit, uint32_t site)
 {
+    if (mbar_try_wait(bar, parity))
+        return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait(bar, parity))
@@ -174,183 +148,323 @@ __device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatil
     }
 }
 
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t *abort,
-                                         unsigned long long limit, uint32_t site)
+// ------------------------------------------------------------------ producers (both CTAs)
+// Two threads of the TMA warp, one per ring.  K(j) and V(j) live in stage
+// j % 2.  Lane 0 loads Q, K(0..1) (barrier k0_full), then K(j+2) once S(j)
+// has completed (s_full), counted on the leader's ready[j % 2]; for the last
+// two steps it only arrives there.  Lane 1 loads V(j) once PV(j-2) has
+// completed (pv_done), counted on ready[j % 2] (bf16) or on this CTA's
+// v_full[j % 2] (FP8: converted first).  s_full / pv_done phases cannot run
+// two ahead of these waits (S(j+2) needs K(j+2), PV(j) needs V(j)).
+template <class C>
+__device__ __forceinline__ void pair_producer(const PairCtx<C> &x, const FwdParams &p, int lane,
+                                              const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                                              const CUtensorMap *tm_v)
 {
-    if (mbar_try_wait(bar, parity))
-        return true;
-    return wait_slow(bar, parity, abort, limit, site);
-}
-
-// Named barrier with an AND-reduction: every participant learns whether all
-// of them are still healthy (keeps later decisions uniform).
-__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t nthreads, bool pred)
-{
-    uint32_t out;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(out)
-        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-        : "memory");
-    return out != 0;
-}
-
-__device__ __forceinline__ float ex2_approx(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ uint32_t pack_p(float lo, float hi, bool f16)
-{
-    if (f16) {
-        __half2 h = __floats2half2_rn(lo, hi);
-        return *reinterpret_cast<uint32_t *>(&h);
+    auto *bars = x.bars;
+    const bool leader = x.rank == 0;
+    const uint64_t pol_kv = l2_policy_evict_last();
+    const uint64_t pol_q = l2_policy_evict_first();
+    const int n = p.n_kv, n0 = n < 2 ? n : 2;
+    bool ok = true;
+    auto k_dst = [&](int j, int b) {
+        return x.base + C::OFF_K + (j % 2) * align_up(C::KTILE, 1024) + b * C::KBOX_BYTES;
+    };
+    if (lane == 0) {
+        if (leader) {
+            mbar_arrive_expect_tx(x.bar(bars->q_full), 2 * C::QTILE);
+            mbar_arrive_expect_tx(x.bar(bars->k0_full), 2 * n0 * C::KTILE);
+        }
+        for (int b = 0; b < C::NBOX; ++b)
+            tma_load_3d_pair(x.base + C::OFF_Q + b * C::QBOX_BYTES, tm_q, x.leader_bar(bars->q_full),
+                             b * C::BOX_ELEMS, x.q0, x.bh, pol_q);
+        for (int j = 0; j < n0; ++j)
+            for (int b = 0; b < C::NBOX; ++b)
+                tma_load_3d_pair(k_dst(j, b), tm_k, x.leader_bar(bars->k0_full), b * C::BOX_ELEMS,
+                                 j * kBN + (int)x.rank * C::KROWS, x.bh, pol_kv);
+        for (int j = 0; j < n && ok; ++j) {
+            const int b2 = j % 2, m = j + 2;            // load K(m) for step j
+            ok = wait_bar_cluster(x.bar(bars->s_full[b2]), (j / 2) & 1, x.abort, x.lim, kSiteKvEmpty);
+            if (!ok)
+                break;
+            if (m < n) {
+                if (leader)
+                    mbar_arrive_expect_tx(x.bar(bars->ready[b2]), 2 * C::KTILE);
+                for (int b = 0; b < C::NBOX; ++b)
+                    tma_load_3d_pair(k_dst(m, b), tm_k, x.leader_bar(bars->ready[b2]), b * C::BOX_ELEMS,
+                                     m * kBN + (int)x.rank * C::KROWS, x.bh, pol_kv);
+            } else if (leader) {
+                mbar_arrive(x.bar(bars->ready[b2]));
+            }
+        }
+    } else if (lane == 1) {
+        for (int j = 0; j < n && ok; ++j) {
+            const int st = j % 2;
+            if (j >= 2)
+                ok = wait_bar_cluster(x.bar(bars->pv_done[st]), ((j - 2) / 2) & 1, x.abort, x.lim, kSiteKvEmpty);
+            if (!ok)
+                break;
+            const uint32_t dst = x.base + C::OFF_V + st * align_up(C::VRAW_TILE, 1024);
+            if (C::FP8) {
+                mbar_arrive_expect_tx(x.bar(bars->v_full[st]), C::VRAW_TILE);
+                tma_load_3d(dst, tm_v, x.bar(bars->v_full[st]), (int)x.rank * (C::D / 2), j * kBN, x.bh, pol_kv);
+            } else {
+                if (leader)
+                    mbar_arrive_expect_tx(x.bar(bars->ready[st]), 2 * C::VRAW_TILE);
+                tma_load_3d_pair(dst, tm_v, x.leader_bar(bars->ready[st]), (int)x.rank * (C::D / 2),
+                                 j * kBN, x.bh, pol_kv);
+            }
+        }
     }
-    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&b);
-}
-
-__device__ __forceinline__ uint32_t cvt_e4m3x2_to_f16x2(uint32_t two_codes)
-{
-    uint32_t r;
-    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
-        : "=r"(r)
-        : "r"(two_codes));
-    return r;
-}
-
-// Byte offset of a 16-byte chunk inside a swizzled tile: the swizzle XORs
-// the chunk bits [4, 4+log2(span/16)) with the row bits [7, ...).
-template <int SPAN>
-__device__ __forceinline__ uint32_t swz(uint32_t off)
-{
-    constexpr uint32_t mask = SPAN == 128 ? 0x70u : (SPAN == 64 ? 0x30u : 0x10u);
-    return off ^ ((off >> 3) & mask);
-}
-
-// ------------------------------------------------------------------ softmax of one S tile
-
-__device__ __forceinline__ float max3f(float a, float b, float c)
-{
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
-// 2^x for a pair, on the FMA/ALU pipes instead of MUFU.  x = n + f with
-// n = rint(x) (adding 1.5*2^23 leaves rint(x) in the low mantissa bits) and
-// f in [-1/2, 1/2]; 2^f is a cubic fitted for minimum max relative error on
-// [-1/2, 1/2] (max rel. error 7.5e-5, below the half-ulp of bf16 and f16 P);
-// 2^n is added to the exponent field.  x is clamped to >= -126 so the
-// exponent never underflows; the callers guarantee x <= 9.
-constexpr float kPolyC0 = 0.9999281167984009f, kPolyC1 = 0.6932609677314758f,
-                kPolyC2 = 0.24261052906513214f, kPolyC3 = 0.05517127364873886f;
-constexpr float kRintMagic = 12582912.0f;   // 1.5 * 2^23
-
-__device__ __forceinline__ float2 exp2_poly2(float2 x)
-{
-    x.x = fmaxf(x.x, -126.f);
-    x.y = fmaxf(x.y, -126.f);
-    const float2 t = __fadd2_rn(x, make_float2(kRintMagic, kRintMagic));
-    const float2 n = __fadd2_rn(t, make_float2(-kRintMagic, -kRintMagic));
-    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-    float2 q = __ffma2_rn(f, make_float2(kPolyC3, kPolyC3), make_float2(kPolyC2, kPolyC2));
-    q = __ffma2_rn(q, f, make_float2(kPolyC1, kPolyC1));
-    q = __ffma2_rn(q, f, make_float2(kPolyC0, kPolyC0));
-    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
-}
-
-// Loads this thread's row of S (128 fp32), updates the running max / sum,
-// writes P (16-bit) over the S columns and rescales O when needed.  P chunk
-// i (S columns 32i..32i+31) goes to columns 16i..16i+15, which hold S values
-// already consumed, so P can be stored chunk by chunk.  Of every 8 element
-// pairs, EMU pairs take 2^x from exp2_poly2 (FMA pipe), the rest from MUFU,
-// which balances the two pipes.
-template <class C, bool MASK, int EMU>
-__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int valid, bool first,
-                                             float c2, float &m_use, float &l)
-{
-    uint32_t s[4][32];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        tmem_ld32(tS + 32 * i, s[i]);
-    tmem_wait_ld();
-
-    if (MASK) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-                if (32 * i + c >= valid)
-                    s[i][c] = __float_as_uint(-INFINITY);
+    if (!ok) {
+        // Give copies already in flight time to land before the cluster exits.
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 20000ull) {
+        }
     }
-    // Row max: 8 independent chains of 3-input max, then a short tree.
+}
+
+// ------------------------------------------------------------------ MMA issuer (leader, one thread)
+template <class C>
+__device__ __forceinline__ void pair_mma(const PairCtx<C> &x, const FwdParams &p)
+{
+    auto *bars = x.bars;
+    constexpr uint16_t kBoth = 0x3;
+    // S(j) into buffer j % 2 from K stage j % 2.
+    auto issue_s = [&](int buf) {
+        const uint32_t q_addr = x.base + C::OFF_Q;
+        const uint32_t k_addr = x.base + C::OFF_K + buf * align_up(C::KTILE, 1024);
+        const uint32_t tS = x.tmem + C::TM_S + 128u * buf;
+#pragma unroll
+        for (int kk = 0; kk < C::QK_STEPS; ++kk) {
+            const uint32_t b = kk / C::STEPS_PER_BOX, w = (kk % C::STEPS_PER_BOX) * C::KSTEP;
+            const uint64_t ad = make_smem_desc(q_addr + b * C::QBOX_BYTES + w, 16, 8 * C::SWZ, C::SWZ_MODE);
+            const uint64_t bd = make_smem_desc(k_addr + b * C::KBOX_BYTES + w, 16, 8 * C::SWZ, C::SWZ_MODE);
+            if (C::FP8)
+                mma2_f8_ss(tS, ad, bd, C::IDESC_QK, kk > 0);
+            else
+                mma2_f16_ss(tS, ad, bd, C::IDESC_QK, kk > 0);
+        }
+    };
+    // PV(j) from buffer j % 2: key half h (P_h, V rows 64h..64h+63) into O_h.
+    auto issue_pv = [&](int buf, uint32_t v_addr, bool first) {
+        const uint32_t tS = x.tmem + C::TM_S + 128u * buf;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int h = m >> 2, kk = m & 3;
+            const uint64_t bd = make_smem_desc(v_addr + (64 * h + 16 * kk) * C::VROW, 16, 8 * C::VROW,
+                                               C::V_SWZ_MODE);
+            mma2_f16_ts(x.tmem + C::TM_O + h * C::D, tS + 64 * h + 8 * kk, bd, C::IDESC_PV,
+                        (first && kk == 0) ? 0u : 1u);
+        }
+    };
+    auto v_operand = [&](int j) {
+        return C::FP8 ? x.base + C::OFF_VH + (j & 1) * align_up(C::VTILE16, 1024)
+                      : x.base + C::OFF_V + (j % 2) * align_up(C::VRAW_TILE, 1024);
+    };
+    bool ok = true;
+    // Everything step j needs (P(j), V(j), K(j+2)) completes one barrier.
+    auto wait_ready = [&](int j) {
+        ok = ok && wait_bar_cluster(x.bar(bars->ready[j % 2]), (j / 2) & 1, x.abort, x.lim, kSitePFull);
+    };
+    const int n = p.n_kv, n0 = n < 2 ? n : 2;
+    ok = wait_bar_cluster(x.bar(bars->q_full), 0, x.abort, x.lim, kSiteQFull) &&
+         wait_bar_cluster(x.bar(bars->k0_full), 0, x.abort, x.lim, kSiteKFull);
+    if (ok) {
+        tc_fence_after();
+        for (int s = 0; s < n0; ++s) {
+            issue_s(s);
+            mma2_commit_mc(x.bar(bars->s_full[s]), kBoth);
+        }
+    }
+    // Per step j: once P(j), V(j) and K(j+2) are in (ready[j % 2]), PV(j) and
+    // then S(j+2) into the same buffer.  S(j+2) depends on nothing of step
+    // j+1, so the softmax of step j+1 overlaps both.
+    for (int j = 0; j < n; ++j) {
+        const int buf = j % 2;
+        wait_ready(j);
+        if (!ok)
+            break;
+        tc_fence_after();
+        issue_pv(buf, v_operand(j), j == 0);
+        mma2_commit_mc(x.bar(bars->pv_done[buf]), kBoth);
+        if (j + 2 < n) {
+            issue_s(buf);
+            mma2_commit_mc(x.bar(bars->s_full[buf]), kBoth);
+        }
+    }
+    if (!ok) {
+        mma2_commit(x.bar(bars->drain));
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(x.bar(bars->drain), 0) && globaltimer_ns() - t0 < 50000000ull) {
+        }
+    }
+}
+
+// ------------------------------------------------------------------ FP8: V half e4m3 -> f16
+template <class C>
+__device__ __forceinline__ void pair_convert_v(const PairCtx<C> &x, const FwdParams &p)
+{
+    auto *bars = x.bars;
+    const int ct = threadIdx.x - C::CONV_WARP0 * 32;
+    constexpr int CPR = C::VRAW_ROW / 16;               // raw 16-byte chunks per key row
+    constexpr int CHUNKS = kBN * CPR;
+    const uint32_t ready_leader[2] = {x.leader_bar(bars->ready[0]), x.leader_bar(bars->ready[1])};
+    for (int j = 0; j < p.n_kv; ++j) {
+        const int st = j % 2;
+        bool ok = wait_bar(x.bar(bars->v_full[st]), (j / 2) & 1, x.abort, x.lim, kSiteConvFull);
+        // f16 buffer j & 1 was last read by PV(j-2).
+        if (j >= 2)
+            ok = ok && wait_bar_cluster(x.bar(bars->pv_done[st]), ((j - 2) / 2) & 1, x.abort, x.lim,
+                                        kSiteVhEmpty);
+        if (!bar_and(6, C::CONV_THREADS, ok))
+            break;
+        const uint32_t src = x.base + C::OFF_V + st * align_up(C::VRAW_TILE, 1024);
+        const uint32_t dst = x.base + C::OFF_VH + (j & 1) * align_up(C::VTILE16, 1024);
+        for (int idx = ct; idx < CHUNKS; idx += C::CONV_THREADS) {
+            const int r = idx / CPR, d0 = (idx % CPR) * 16;
+            uint32_t w[4];
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "r"(src + swz<C::VRAW_ROW>((uint32_t)(r * C::VRAW_ROW + d0))));
+            uint32_t hv[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                hv[2 * i] = cvt_e4m3x2_to_f16x2(w[i] & 0xFFFFu);
+                hv[2 * i + 1] = cvt_e4m3x2_to_f16x2(w[i] >> 16);
+            }
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const uint32_t off = swz<C::VROW>((uint32_t)(r * C::VROW + (d0 + 8 * half) * 2));
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + off),
+                             "r"(hv[4 * half]), "r"(hv[4 * half + 1]), "r"(hv[4 * half + 2]),
+                             "r"(hv[4 * half + 3])
+                             : "memory");
+            }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(6, C::CONV_THREADS);
+        if (ct == 0)
+            mbar_arrive_cluster(ready_leader[j % 2]);
+    }
+}
+
+// ------------------------------------------------------------------ softmax (two threads per row)
+
+// Max of this thread's 64 S values (keys >= valid count as -inf).
+template <bool MASK>
+__device__ __forceinline__ float half_row_max(const uint32_t (&s)[2][32], int kbase, int valid)
+{
+    auto val = [&](int i, int c) {
+        const float v = __uint_as_float(s[i][c]);
+        return (!MASK || kbase + 32 * i + c < valid) ? v : -INFINITY;
+    };
     float m8[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-        m8[k] = fmaxf(__uint_as_float(s[0][2 * k]), __uint_as_float(s[0][2 * k + 1]));
+        m8[k] = fmaxf(val(0, 2 * k), val(0, 2 * k + 1));
 #pragma unroll
-    for (int e = 16; e < 128; e += 16)
+    for (int e = 16; e < 64; e += 16)
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-            m8[k] = max3f(m8[k], __uint_as_float(s[e >> 5][(e & 31) + 2 * k]),
-                          __uint_as_float(s[e >> 5][(e & 31) + 2 * k + 1]));
-    const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+            m8[k] = max3f(m8[k], val(e >> 5, (e & 31) + 2 * k), val(e >> 5, (e & 31) + 2 * k + 1));
+    return max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+}
 
-    float alpha = 1.f;
-    if (first) {
-        m_use = mx;
-    } else if ((mx - m_use) * c2 > kRescaleLog2) {
-        alpha = ex2_approx((m_use - mx) * c2);
-        m_use = mx;
-    }
-    const float mc = m_use * c2;
+// p = 2^(s*c2 - mc) for this thread's 64 values, packed to 16 bits and stored
+// as 32 TMEM columns at tS (over S values only this thread has read).
+// Returns the sum of the p.  Of every 8 pairs, EMU use the FMA-pipe exp2.
+template <class C, bool MASK, int EMU>
+__device__ __forceinline__ float half_row_exp_store(const uint32_t (&s)[2][32], uint32_t tS, int kbase, int valid,
+                                                    float c2, float mc)
+{
     const float2 c2c2 = make_float2(c2, c2), nmc = make_float2(-mc, -mc);
-
     float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                      make_float2(0.f, 0.f)};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-            const int pi = (32 * i + c) >> 1;     // pair index 0..63
-            const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[i][c]), __uint_as_float(s[i][c + 1])),
-                                        c2c2, nmc);
+            const int pi = (32 * i + c) >> 1;
+            const float2 xv = __ffma2_rn(make_float2(__uint_as_float(s[i][c]), __uint_as_float(s[i][c + 1])),
+                                         c2c2, nmc);
             float2 e;
             if ((pi & 7) >= 8 - EMU) {
-                e = exp2_poly2(x);
+                e = exp2_poly2(xv);
             } else {
-                e.x = ex2_approx(x.x);
-                e.y = ex2_approx(x.y);
+                e.x = ex2_approx(xv.x);
+                e.y = ex2_approx(xv.y);
             }
             if (MASK) {
-                e.x = (32 * i + c < valid) ? e.x : 0.f;
-                e.y = (32 * i + c + 1 < valid) ? e.y : 0.f;
+                e.x = (kbase + 32 * i + c < valid) ? e.x : 0.f;
+                e.y = (kbase + 32 * i + c + 1 < valid) ? e.y : 0.f;
             }
             acc[pi & 3] = __fadd2_rn(acc[pi & 3], e);
             pk[c / 2] = pack_p(e.x, e.y, C::FP8);
         }
         tmem_st16(tS + 16 * i, pk);
     }
-    const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
-    const float2 a = __fadd2_rn(a01, a23);
-    l = l * alpha + (a.x + a.y);
+    const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+    return a.x + a.y;
+}
 
-    // After the exponentials (S registers dead).  O is stable here: S_g(j)
-    // complete implies PV_g(j-1) complete.
-    if (!first && __any_sync(0xffffffffu, alpha != 1.f)) {
+// Per-thread softmax state: running max (raw S units, lazily raised), running
+// sum of this thread's key half, log2(e) * scale (with the FP8 dequant scales).
+struct HalfRowState {
+    float m_use, l, c2;
+    bool alive;
+};
+
+// One step j for one thread: its 64 values of S(j) -> P(j) (in place in TMEM),
+// running max / sum, lazy rescale of O_h; hands P(j) to the MMA through the
+// leader's ready[j % 2].
+template <class C>
+__device__ __forceinline__ void half_row_step(const PairCtx<C> &x, const FwdParams &p, int j, int h,
+                                              int lane, uint32_t lane_off, uint32_t ready_leader,
+                                              HalfRowState &st)
+{
+    constexpr int D = C::D;
+    auto *bars = x.bars;
+    const int n = p.n_kv, buf = j % 2;
+    st.alive = __all_sync(0xffffffffu, st.alive && wait_bar_cluster(x.bar(bars->s_full[buf]), (j / 2) & 1,
+                                                                     x.abort, x.lim, kSiteSFull));
+    if (!st.alive)
+        return;
+    tc_fence_after();
+    const uint32_t tS = x.tmem + lane_off + C::TM_S + 128u * buf + 64 * h;
+    uint32_t s[2][32];
+    tmem_ld32(tS, s[0]);
+    tmem_ld32(tS + 32, s[1]);
+    tmem_wait_ld_regs(s[0]);
+    tmem_wait_ld_regs(s[1]);
+    const bool masked = j == n - 1 && p.kv_tail < kBN;
+    const float mx = masked ? half_row_max<true>(s, 64 * h, p.kv_tail) : half_row_max<false>(s, 64 * h, kBN);
+    float alpha = 1.f;
+    if (j == 0) {
+        st.m_use = mx;
+    } else if ((mx - st.m_use) * st.c2 > kRescaleLog2) {
+        alpha = ex2_approx((st.m_use - mx) * st.c2);
+        st.m_use = mx;
+    }
+    const float mc = st.m_use * st.c2;
+    const float sum = masked ? half_row_exp_store<C, true, C::EXP_EMU>(s, tS, 64 * h, p.kv_tail, st.c2, mc)
+                             : half_row_exp_store<C, false, C::EXP_EMU>(s, tS, 64 * h, kBN, st.c2, mc);
+    st.l = st.l * alpha + sum;
+    if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // Rescale this thread's row of O_h once PV(j-1) has finished with it.
+        const int jp = j - 1;
+        st.alive = __all_sync(0xffffffffu, wait_bar_cluster(x.bar(bars->pv_done[jp % 2]), (jp / 2) & 1,
+                                                             x.abort, x.lim, kSiteOFull));
+        if (!st.alive)
+            return;
+        tc_fence_after();
+        const uint32_t tO = x.tmem + lane_off + C::TM_O + h * D;
 #pragma unroll
-        for (int cc = 0; cc < C::D / 32; ++cc) {
+        for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
             tmem_ld32(tO + 32 * cc, o);
-            tmem_wait_ld();
+            tmem_wait_ld_regs(o);
 #pragma unroll
             for (int c = 0; c < 32; ++c)
                 o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
@@ -358,297 +472,97 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int valid
         }
     }
     tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive_cluster(ready_leader);
 }
 
-// ------------------------------------------------------------------ roles
-// Shared state every role sees.
 template <class C>
-struct Ctx {
-    Bars<C::NSTAGE> *bars;
-    uint32_t base;                 // 1024-aligned shared-memory base address
-    uint32_t tmem;                 // TMEM base address
-    volatile uint32_t *abort;      // CTA-wide abort flag
-    unsigned long long lim;        // wait limit, ns
-    int bh, q0;                    // (b, h) index and first query row of the pair
-    __device__ uint32_t bar(const uint64_t &b) const { return smem_u32(&b); }
-};
-
-// TMA producer (one thread): both Q tiles once, then K_j, V_j into the ring.
-template <class C>
-__device__ __forceinline__ void producer_role(const Ctx<C> &x, const FwdParams &p,
-                                              const CUtensorMap *tm_q, const CUtensorMap *tm_k,
-                                              const CUtensorMap *tm_v)
-{
-    constexpr int NS = C::NSTAGE;
-    auto *bars = x.bars;
-    const uint64_t pol_kv = l2_policy_evict_last();
-    const uint64_t pol_q = l2_policy_evict_first();
-    mbar_arrive_expect_tx(x.bar(bars->q_full), 2 * C::TILE);
-    for (int g = 0; g < 2; ++g)
-        for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d(x.base + C::OFF_Q + g * C::TILE + b * C::BOX_BYTES, tm_q, x.bar(bars->q_full),
-                        b * C::BOX_ELEMS, x.q0 + g * kBM, x.bh, pol_q);
-    int last_round[NS];
-#pragma unroll
-    for (int s = 0; s < NS; ++s)
-        last_round[s] = -1;
-    const int n_loads = 2 * p.n_kv;
-    for (int t = 0; t < n_loads; ++t) {
-        const int st = t % NS, rd = t / NS;
-        if (!wait_bar(x.bar(bars->kv_empty[st]), (rd & 1) ^ 1, x.abort, x.lim, kSiteKvEmpty))
-            break;
-        const uint32_t fb = x.bar(bars->kv_full[st]);
-        mbar_arrive_expect_tx(fb, C::TILE);
-        const CUtensorMap *m = (t & 1) ? tm_v : tm_k;
-        for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d(x.base + C::OFF_KV + st * C::TILE + b * C::BOX_BYTES, m, fb, b * C::BOX_ELEMS,
-                        (t >> 1) * kBN, x.bh, pol_kv);
-#pragma unroll
-        for (int s = 0; s < NS; ++s)
-            if (s == st)
-                last_round[s] = rd;
-    }
-    if (*x.abort) {
-        // Let copies already in flight land before the CTA exits (bounded).
-        constexpr unsigned long long kDrainNs = 50000000ull;
-#pragma unroll
-        for (int s = 0; s < NS; ++s) {
-            if (last_round[s] < 0)
-                continue;
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(x.bar(bars->kv_full[s]), last_round[s] & 1) &&
-                   globaltimer_ns() - t0 < kDrainNs) {
-            }
-        }
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(x.bar(bars->q_full), 0) && globaltimer_ns() - t0 < kDrainNs) {
-        }
-    }
-}
-
-// MMA issuer (one thread).  Issue order per K/V tile j:
-//   PV0(j), S0(j+1), PV1(j), S1(j+1)   after the prologue S0(0), S1(0).
-template <class C>
-__device__ __forceinline__ void mma_role(const Ctx<C> &x, const FwdParams &p)
-{
-    constexpr int NS = C::NSTAGE;
-    auto *bars = x.bars;
-    auto issue_s = [&](int g, uint32_t k_addr) {
-        const uint32_t q_addr = x.base + C::OFF_Q + g * C::TILE;
-        const uint32_t tS = x.tmem + (g ? C::TM_S1 : C::TM_S0);
-#pragma unroll
-        for (int kk = 0; kk < C::QK_STEPS; ++kk) {
-            const uint32_t off =
-                (kk / C::STEPS_PER_BOX) * C::BOX_BYTES + (kk % C::STEPS_PER_BOX) * C::KSTEP;
-            const uint64_t ad = make_smem_desc(q_addr + off, 16, 8 * C::SWZ, C::SWZ_MODE);
-            const uint64_t bd = make_smem_desc(k_addr + off, 16, 8 * C::SWZ, C::SWZ_MODE);
-            if (C::FP8)
-                mma_f8_ss(tS, ad, bd, C::IDESC_QK, kk > 0);
-            else
-                mma_f16_ss(tS, ad, bd, C::IDESC_QK, kk > 0);
-        }
-    };
-    auto issue_pv = [&](int g, uint32_t v_addr, bool acc) {
-        const uint32_t tS = x.tmem + (g ? C::TM_S1 : C::TM_S0);
-        const uint32_t tO = x.tmem + (g ? C::TM_O1 : C::TM_O0);
-#pragma unroll
-        for (int kk = 0; kk < C::PV_STEPS; ++kk) {
-            const uint64_t bd =
-                make_smem_desc(v_addr + kk * 16 * 128, C::VBOX_BYTES, 1024, kSwizzle128B);
-            mma_f16_ts(tO, tS + kk * 8, bd, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
-        }
-    };
-
-    bool ok = wait_bar(x.bar(bars->q_full), 0, x.abort, x.lim, kSiteQFull) &&
-              wait_bar(x.bar(bars->kv_full[0]), 0, x.abort, x.lim, kSiteKFull);
-    if (ok) {
-        tc_fence_after();
-        const uint32_t k_addr = x.base + C::OFF_KV;
-        issue_s(0, k_addr);
-        mma_commit(x.bar(bars->s_full[0]));
-        issue_s(1, k_addr);
-        mma_commit(x.bar(bars->s_full[1]));
-        mma_commit(x.bar(bars->kv_empty[0]));
-    }
-    for (int j = 0; ok && j < p.n_kv; ++j) {
-        const bool has_next = j + 1 < p.n_kv;
-        uint32_t v_addr;
-        int sv = 0;
-        if (C::FP8) {
-            ok = wait_bar(x.bar(bars->vh_full[j & 1]), (j >> 1) & 1, x.abort, x.lim, kSiteVhFull);
-            v_addr = x.base + C::OFF_VH + (j & 1) * C::VTILE;
-        } else {
-            const int t = 2 * j + 1;
-            sv = t % NS;
-            ok = wait_bar(x.bar(bars->kv_full[sv]), (t / NS) & 1, x.abort, x.lim, kSiteKFull);
-            v_addr = x.base + C::OFF_KV + sv * C::TILE;
-        }
-        int sk = 0;
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-            ok = ok && wait_bar(x.bar(bars->p_full[g]), j & 1, x.abort, x.lim, kSitePFull);
-            if (!ok)
-                break;
-            tc_fence_after();
-            issue_pv(g, v_addr, j > 0);
-            if (!has_next)
-                mma_commit(x.bar(bars->o_full[g]));
-            if (g == 1)
-                mma_commit(C::FP8 ? x.bar(bars->vh_empty[j & 1]) : x.bar(bars->kv_empty[sv]));
-            if (has_next) {
-                if (g == 0) {
-                    const int t = 2 * (j + 1);
-                    sk = t % NS;
-                    ok = wait_bar(x.bar(bars->kv_full[sk]), (t / NS) & 1, x.abort, x.lim, kSiteKFull);
-                    if (!ok)
-                        break;
-                    tc_fence_after();
-                }
-                issue_s(g, x.base + C::OFF_KV + sk * C::TILE);
-                mma_commit(x.bar(bars->s_full[g]));
-                if (g == 1)
-                    mma_commit(x.bar(bars->kv_empty[sk]));
-            }
-        }
-    }
-    if (!ok) {
-        // Wait (bounded) until every MMA issued so far has finished.
-        mma_commit(x.bar(bars->drain));
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(x.bar(bars->drain), 0) && globaltimer_ns() - t0 < 50000000ull) {
-        }
-    }
-}
-
-// FP8 path (warps 10-11): converts each e4m3 V tile of the ring into a
-// 16-bit (f16) MN-major 128B-swizzled tile for the PV MMA, then releases the
-// ring stage.  e4m3 values are exact in f16.
-template <class C>
-__device__ __forceinline__ void convert_v_role(const Ctx<C> &x, const FwdParams &p)
-{
-    constexpr int NS = C::NSTAGE;
-    auto *bars = x.bars;
-    const int ct = threadIdx.x - C::CONV_WARP0 * 32;   // 0..63
-    constexpr int CHUNKS = kBN * C::ROW / 16;          // raw 16-byte chunks per V tile
-    for (int j = 0; j < p.n_kv; ++j) {
-        const int t = 2 * j + 1, st = t % NS;
-        bool ok = wait_bar(x.bar(bars->kv_full[st]), (t / NS) & 1, x.abort, x.lim, kSiteConvFull);
-        ok = ok && wait_bar(x.bar(bars->vh_empty[j & 1]), ((j >> 1) & 1) ^ 1, x.abort, x.lim,
-                            kSiteVhEmpty);
-        if (!bar_and(3, C::CONV_THREADS, ok))
-            break;
-        const uint32_t src = x.base + C::OFF_KV + st * C::TILE;
-        const uint32_t dst = x.base + C::OFF_VH + (j & 1) * C::VTILE;
-        for (int idx = ct; idx < CHUNKS; idx += C::CONV_THREADS) {
-            const int r = idx / (C::ROW / 16);      // key row
-            const int d0 = (idx % (C::ROW / 16)) * 16;  // first of 16 elements
-            const uint32_t roff = (d0 / C::BOX_ELEMS) * C::BOX_BYTES +
-                                  swz<C::SWZ>((uint32_t)r * C::SWZ + (uint32_t)(d0 % C::BOX_ELEMS));
-            uint32_t w[4];
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                         : "r"(src + roff));
-            uint32_t h[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                h[2 * i] = cvt_e4m3x2_to_f16x2(w[i] & 0xFFFFu);
-                h[2 * i + 1] = cvt_e4m3x2_to_f16x2(w[i] >> 16);
-            }
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int d = d0 + 8 * half;        // 8 f16 = one 16-byte chunk
-                const uint32_t doff =
-                    (d / 64) * C::VBOX_BYTES + swz<128>((uint32_t)r * 128u + (uint32_t)(d % 64) * 2u);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + doff),
-                             "r"(h[4 * half]), "r"(h[4 * half + 1]), "r"(h[4 * half + 2]),
-                             "r"(h[4 * half + 3])
-                             : "memory");
-            }
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(3, C::CONV_THREADS);
-        if (ct == 0) {
-            mbar_arrive(x.bar(bars->vh_full[j & 1]));
-            mbar_arrive(x.bar(bars->kv_empty[st]));
-        }
-    }
-}
-
-// Softmax + epilogue of query tile g (warps 4g..4g+3, one thread per row).
-template <class C>
-__device__ __forceinline__ void softmax_role(const Ctx<C> &x, const FwdParams &p,
+__device__ __forceinline__ void pair_softmax(const PairCtx<C> &x, const FwdParams &p,
                                              const CUtensorMap *tm_o, int warp, int lane)
 {
     constexpr int D = C::D;
     auto *bars = x.bars;
-    const int g = warp >> 2;
-    const int wq = warp & 3;             // TMEM lane quarter this warp may access
-    const int row = wq * 32 + lane;      // row inside query tile g
+    const int h = warp >> 2, wq = warp & 3;
+    const int row = wq * 32 + lane;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = x.tmem + lane_off + (g ? C::TM_S1 : C::TM_S0);
-    const uint32_t tO = x.tmem + lane_off + (g ? C::TM_O1 : C::TM_O0);
-    float c2 = p.scale * kLog2e;         // logit scale in log2 units
+    float *red = reinterpret_cast<float *>(x.sm + C::OFF_RED);
+    const uint32_t bar_id = 1 + wq;
+    const uint32_t ready_leader[2] = {x.leader_bar(bars->ready[0]), x.leader_bar(bars->ready[1])};
+    HalfRowState st;
+    st.c2 = p.scale * kLog2e;
     float vs = 1.f;
     if (C::FP8) {
-        c2 = p.scale * p.q_scale[x.bh] * p.k_scale[x.bh] * kLog2e;
+        st.c2 = p.scale * p.q_scale[x.bh] * p.k_scale[x.bh] * kLog2e;
         vs = p.v_scale[x.bh];
     }
-    float m_use = -INFINITY, l = 0.f;
-    bool alive = true;
-    for (int j = 0; j < p.n_kv; ++j) {
-        const bool ok = wait_bar(x.bar(bars->s_full[g]), j & 1, x.abort, x.lim, kSiteSFull);
-        if (!__all_sync(0xffffffffu, ok)) {
-            alive = false;
-            break;
-        }
-        tc_fence_after();
-        if (j + 1 < p.n_kv || p.kv_tail == kBN)
-            softmax_tile<C, false, C::EXP_EMU>(tS, tO, kBN, j == 0, c2, m_use, l);
-        else
-            softmax_tile<C, true, C::EXP_EMU>(tS, tO, p.kv_tail, j == 0, c2, m_use, l);
-        tc_fence_before();
-        mbar_arrive(x.bar(bars->p_full[g]));
+    st.m_use = -INFINITY;
+    st.l = 0.f;
+    st.alive = true;
+    const int n = p.n_kv;
+    for (int j = 0; j < n && st.alive; j += 2) {
+        half_row_step<C>(x, p, j, h, lane, lane_off, ready_leader[0], st);
+        if (j + 1 < n && st.alive)
+            half_row_step<C>(x, p, j + 1, h, lane, lane_off, ready_leader[1], st);
     }
-    // ---- epilogue: O / l -> bf16 -> swizzled staging smem -> TMA store; LSE.
-    if (alive)
-        alive = __all_sync(0xffffffffu,
-                           wait_bar(x.bar(bars->o_full[g]), 0, x.abort, x.lim, kSiteOFull));
-    const uint32_t ost =
-        C::FP8 ? x.base + C::OFF_OST + g * C::OTILE : x.base + C::OFF_Q + g * C::TILE;
+    bool alive = st.alive;
+    // ---- epilogue: merge the two key halves through their log-sum-exp,
+    // (a_0 O_0 + a_1 O_1) / l -> bf16 -> staging -> TMA store; LSE.
+    if (alive) {
+        const int jl = n - 1;
+        alive = __all_sync(0xffffffffu, wait_bar_cluster(x.bar(bars->pv_done[jl % 2]), (jl / 2) & 1, x.abort,
+                                                          x.lim, kSiteOFull));
+    }
+    // A half with no valid key (L < 64) has l = 0 and takes no part.
+    const float m2 = st.l > 0.f ? st.m_use * st.c2 : -INFINITY;
+    red[h * kBM + row] = m2;
+    red[(2 + h) * kBM + row] = st.l;
+    alive = bar_and(bar_id, 64, alive);
+    const float m2o = red[(1 - h) * kBM + row], lo = red[(3 - h) * kBM + row];
+    const float mrow = fmaxf(m2, m2o);
+    const float a_self = ex2_approx(m2 - mrow), a_other = ex2_approx(m2o - mrow);
+    const float l_row = st.l * a_self + lo * a_other;
+    const float a0 = h == 0 ? a_self : a_other, a1 = h == 0 ? a_other : a_self;
+    const uint32_t ost = C::FP8 ? x.base + C::OFF_OST : x.base + C::OFF_Q;
     if (alive) {
         tc_fence_after();
-        const float inv = vs / l;
+        const float inv = vs / l_row;
+        const float w0 = a0 * inv, w1 = a1 * inv;
+        // This thread writes output columns h*D/2 .. h*D/2 + D/2 of its row.
+        const uint32_t tO0 = x.tmem + lane_off + C::TM_O + h * (D / 2);
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * cc, o);
-            tmem_wait_ld();
+        for (int cc = 0; cc < D / 64; ++cc) {
+            uint32_t o0[32], o1[32];
+            tmem_ld32(tO0 + 32 * cc, o0);
+            tmem_ld32(tO0 + D + 32 * cc, o1);
+            tmem_wait_ld_regs(o0);
+            tmem_wait_ld_regs(o1);
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-                pk[i] = pack_p(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv,
-                               false);
+                pk[i] = pack_p(__uint_as_float(o0[2 * i]) * w0 + __uint_as_float(o1[2 * i]) * w1,
+                               __uint_as_float(o0[2 * i + 1]) * w0 + __uint_as_float(o1[2 * i + 1]) * w1, false);
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
-                const int chunk = 4 * cc + k4;   // 16-byte chunk of this row
+                const int chunk = h * (D / 16) + 4 * cc + k4;     // 16-byte chunk of the output row
                 const uint32_t off = (chunk >> 3) * C::OBOX_BYTES +
                                      swz<128>((uint32_t)row * 128u + (uint32_t)(chunk & 7) * 16u);
                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ost + off),
-                             "r"(pk[4 * k4]), "r"(pk[4 * k4 + 1]), "r"(pk[4 * k4 + 2]),
-                             "r"(pk[4 * k4 + 3])
+                             "r"(pk[4 * k4]), "r"(pk[4 * k4 + 1]), "r"(pk[4 * k4 + 2]), "r"(pk[4 * k4 + 3])
                              : "memory");
             }
         }
         fence_proxy_async_smem();
     }
-    alive = bar_and(1 + g, 128, alive);
+    alive = bar_and(5, 256, alive);
     if (alive) {
-        const int qrow = x.q0 + g * kBM + row;
-        if (p.lse != nullptr && qrow < p.L)
-            p.lse[(long long)x.bh * p.L + qrow] = (m_use * c2 + log2f(l)) * kLn2;
-        if (row == 0) {
+        const int qrow = x.q0 + row;
+        if (h == 0 && p.lse != nullptr && qrow < p.L)
+            p.lse[(long long)x.bh * p.L + qrow] = (mrow + log2f(l_row)) * kLn2;
+        if (warp == 0 && lane == 0) {
             for (int b = 0; b < C::OBOX; ++b)
-                tma_store_3d(tm_o, ost + b * C::OBOX_BYTES, b * 64, x.q0 + g * kBM, x.bh);
+                tma_store_3d(tm_o, ost + b * C::OBOX_BYTES, b * 64, x.q0, x.bh);
             bulk_commit_group();
             bulk_wait_group_all();
         }
@@ -656,36 +570,29 @@ __device__ __forceinline__ void softmax_role(const Ctx<C> &x, const FwdParams &p
 }
 
 // ------------------------------------------------------------------ the kernel
-
 template <int D, bool FP8>
-__global__ void __launch_bounds__(KCfg<D, FP8>::THREADS, 1)
+__global__ void __launch_bounds__(PCfg<D, FP8>::THREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                const FwdParams p)
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                     const FwdParams p)
 {
-    using C = KCfg<D, FP8>;
-    constexpr int NS = C::NSTAGE;
+    using C = PCfg<D, FP8>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
-    Bars<NS> *bars = reinterpret_cast<Bars<NS> *>(smem_raw + (base - raw_addr) + C::OFF_BAR);
+    PairBars *bars = reinterpret_cast<PairBars *>(smem_raw + (base - raw_addr) + C::OFF_BAR);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
 
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-
-    // ---- set-up: barriers (one thread), TMEM (MMA warp)
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bars->q_full), 1);
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(smem_u32(&bars->kv_full[s]), 1);
-            mbar_init(smem_u32(&bars->kv_empty[s]), 1);
-        }
-        for (int g = 0; g < 2; ++g) {
-            mbar_init(smem_u32(&bars->s_full[g]), 1);
-            mbar_init(smem_u32(&bars->p_full[g]), kBM);
-            mbar_init(smem_u32(&bars->o_full[g]), 1);
-            mbar_init(smem_u32(&bars->vh_full[g]), 1);
-            mbar_init(smem_u32(&bars->vh_empty[g]), 1);
+        mbar_init(smem_u32(&bars->k0_full), 1);
+        // ready: 16 softmax warps + the K producer + (bf16) the V producer or (FP8) two converters.
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&bars->ready[b]), FP8 ? 19 : 18);
+            mbar_init(smem_u32(&bars->v_full[b]), 1);
+            mbar_init(smem_u32(&bars->s_full[b]), 1);
+            mbar_init(smem_u32(&bars->pv_done[b]), 1);
         }
         mbar_init(smem_u32(&bars->drain), 1);
         bars->abort = 0u;
@@ -699,65 +606,50 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tma_prefetch_desc(&tm_o);
     }
     if (warp == C::MMA_WARP) {
-        tmem_alloc(smem_u32(&bars->tmem_base), C::TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_u32(&bars->tmem_base), C::TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
 
-    Ctx<C> x;
+    PairCtx<C> x;
     x.bars = bars;
+    x.sm = smem_raw + (base - raw_addr);
     x.base = base;
     x.tmem = bars->tmem_base;
+    x.rank = rank;
     x.abort = &bars->abort;
     x.lim = p.wait_limit_ns;
-    x.bh = blockIdx.x / p.n_pairs;
-    x.q0 = (blockIdx.x % p.n_pairs) * 2 * kBM;
+    const int cluster = blockIdx.x >> 1;
+    x.bh = cluster / p.n_pairs;
+    x.q0 = (cluster % p.n_pairs) * 2 * kBM + (int)rank * kBM;
 
     if (warp >= 8) {
-        // Warpgroup 2: producer, MMA issuer, converter.  Each warpgroup sets
-        // its register budget at the top of its own branch.
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
         if (warp == C::TMA_WARP) {
-            if (lane == 0)
-                producer_role<C>(x, p, &tm_q, &tm_k, &tm_v);
+            if (lane < 2)
+                pair_producer<C>(x, p, lane, &tm_q, &tm_k, &tm_v);
         } else if (warp == C::MMA_WARP) {
-            if (lane == 0)
-                mma_role<C>(x, p);
+            if (lane == 0 && rank == 0)
+                pair_mma<C>(x, p);
         } else if (FP8) {
-            convert_v_role<C>(x, p);
+            pair_convert_v<C>(x, p);
         }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFTMAX));
-        softmax_role<C>(x, p, &tm_o, warp, lane);
+        pair_softmax<C>(x, p, &tm_o, warp, lane);
     }
 
-    // ---- tear-down
+    // Neither CTA leaves (or frees TMEM) while the pair's MMAs may still touch it.
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     if (warp == C::MMA_WARP) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(x.tmem, C::TMEM_COLS);
+        tmem_dealloc_pair(x.tmem, C::TMEM_COLS);
     }
-}
-
-// Self-test of the bounded wait: one thread waits on an mbarrier nothing completes.
-__global__ void selftest_wait_kernel(unsigned long long limit_ns)
-{
-    __shared__ uint64_t bar;
-    __shared__ uint32_t abort;
-    if (threadIdx.x == 0) {
-        mbar_init(smem_u32(&bar), 1);
-        abort = 0u;
-        fence_barrier_init();
-    }
-    __syncthreads();
-    if (threadIdx.x == 0)
-        wait_bar(smem_u32(&bar), 0, reinterpret_cast<volatile uint32_t *>(&abort), limit_ns,
-                 kSiteSelftest);
-    __syncthreads();
 }
 
 } // namespace dit

@@ -32,55 +32,71 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// 3-D map over a contiguous [BH, L, D] tensor: dims (D, L, BH), box (box_x, 128, 1).
+// 3-D map over a contiguous [BH, L, D] tensor: dims (D, L, BH), box (box_x, box_rows, 1).
 bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int elt, int D, int L,
-              long long BH, int box_x, CUtensorMapSwizzle swz)
+              long long BH, int box_x, CUtensorMapSwizzle swz, int box_rows = dit::kBM)
 {
     auto enc = tensor_map_encoder();
     if (!enc)
         return false;
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)BH};
     const cuuint64_t strides[2] = {(cuuint64_t)D * elt, (cuuint64_t)L * D * elt};
-    const cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)dit::kBM, 1u};
+    const cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_rows, 1u};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
     return enc(m, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+CUtensorMapSwizzle swizzle_for(int bytes)
+{
+    return bytes >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B : (bytes >= 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
 // Per-device "max dynamic smem attribute set" flags, one per kernel instantiation.
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_attr_set[4][kMaxDevices];
 
+// Clusters of 2 CTAs, one 128-row query tile per CTA.
 template <int D, bool FP8>
 int launch(const void *q, const void *k, const void *v, void *o, const dit::FwdParams &prm,
-           long long BH, int L, int device, cudaStream_t stream)
+                long long BH, int L, int device, cudaStream_t stream)
 {
-    using C = dit::KCfg<D, FP8>;
+    using C = dit::PCfg<D, FP8>;
     constexpr int variant = (D == 128 ? 1 : 0) + (FP8 ? 2 : 0);
     auto kern = dit::attn_fwd_kernel<D, FP8>;
-    if (device < kMaxDevices && g_attr_set[variant][device].load(std::memory_order_acquire) == 0) {
+    if (device >= kMaxDevices || g_attr_set[variant][device].load(std::memory_order_acquire) == 0) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
             cudaSuccess)
             return DIT_ATTN_ERR_LAUNCH;
-        g_attr_set[variant][device].store(1, std::memory_order_release);
-    } else if (device >= kMaxDevices) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-            cudaSuccess)
-            return DIT_ATTN_ERR_LAUNCH;
+        if (device < kMaxDevices)
+            g_attr_set[variant][device].store(1, std::memory_order_release);
     }
     const CUtensorMapDataType in_t = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const CUtensorMapSwizzle in_swz = C::SWZ == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap tq, tk, tv, to;
-    if (!make_map(&tq, q, in_t, C::ELT, D, L, BH, C::BOX_ELEMS, in_swz) ||
-        !make_map(&tk, k, in_t, C::ELT, D, L, BH, C::BOX_ELEMS, in_swz) ||
-        !make_map(&tv, v, in_t, C::ELT, D, L, BH, C::BOX_ELEMS, in_swz) ||
-        !make_map(&to, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, L, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_map(&tq, q, in_t, C::ELT, D, L, BH, C::BOX_ELEMS, swizzle_for(C::SWZ), dit::kBM) ||
+        !make_map(&tk, k, in_t, C::ELT, D, L, BH, C::BOX_ELEMS, swizzle_for(C::SWZ), C::KROWS) ||
+        !make_map(&tv, v, in_t, C::ELT, D, L, BH, D / 2, swizzle_for(C::VRAW_ROW), dit::kBN) ||
+        !make_map(&to, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, L, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+                  dit::kBM))
         return DIT_ATTN_ERR_LAUNCH;
-    const long long blocks = BH * (long long)prm.n_pairs;
+    const long long blocks = 2 * BH * (long long)prm.n_pairs;
     if (blocks > 0x7FFFFFFFll)
         return DIT_ATTN_ERR_SHAPE;
-    kern<<<dim3((unsigned)blocks), dim3(C::THREADS), C::SMEM_BYTES, stream>>>(tq, tk, tv, to, prm);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, prm) != cudaSuccess)
+        return DIT_ATTN_ERR_LAUNCH;
     return cudaGetLastError() == cudaSuccess ? DIT_ATTN_OK : DIT_ATTN_ERR_LAUNCH;
 }
 

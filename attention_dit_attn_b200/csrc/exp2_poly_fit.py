@@ -1,4 +1,4 @@
-"""Fits the cubic used by the kernel's FMA-pipe exp2 (exp2_poly2 in attn_fwd_sm100.cuh).
+"""Fits the cubic used by the kernel's FMA-pipe exp2 (exp2_poly2 in attn_common.cuh).
 
 2^x is split as 2^n * 2^f with n = rint(x), f in [-1/2, 1/2]; 2^f is approximated
 by c0 + c1 f + c2 f^2 + c3 f^3 with coefficients chosen to minimise the maximum

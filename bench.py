@@ -409,7 +409,7 @@ def run_ours(args, dist: Dist):
         "gpu_launches": launches,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "peak_source": peak_note, "traffic": traffic,
-                     "kernel": "dit::attn_fwd_kernel", "flops_per_launch": w.flops},
+                     "kernel": "dit::attn_fwd_kernel (CTA pair)", "flops_per_launch": w.flops},
         "clocks": clocks,
     }
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:

@@ -13,7 +13,7 @@ import exp2_poly_fit  # noqa: E402
 
 
 def kernel_coeffs():
-    text = open(os.path.join(CSRC, "attn_fwd_sm100.cuh")).read()
+    text = open(os.path.join(CSRC, "attn_common.cuh")).read()
     vals = {k: float(v) for k, v in re.findall(r"kPolyC(\d) = ([0-9.eE+-]+)f", text)}
     return np.array([vals["0"], vals["1"], vals["2"], vals["3"]], dtype=np.float32)
 
