@@ -27,6 +27,18 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f; // lazy-rescale threshold (p <= 256)
 
+// bf16 P is the high half of the f32 p (one byte permute, i.e. truncation).
+// That drops 16 mantissa bits: on average over the dropped bits the loss is
+// 2^-8 / (1+m) of p, where 1+m is p's significand.  For p = 2^x with x spread
+// over many units, 1+m is log-uniform on [1, 2), where E[1/(1+m)] =
+// 1/(2 ln 2), so the mean relative loss is mu = 1/(512 ln 2) = 2.818e-3.
+// Every p is computed as p * kTruncGain, kTruncGain = 1/(1 - mu) (an offset
+// of kTruncLog2 on the exponent), which makes the truncated value unbiased;
+// the running sums then carry the same factor, which the epilogue takes out of
+// O and the LSE.
+constexpr float kTruncGain = 1.0028257f;
+constexpr float kTruncLog2 = 0.0040709f;   // log2(kTruncGain)
+
 // Wait sites recorded in the error word (bits 8..15).
 enum : uint32_t {
     kSiteQFull = 1, kSiteKFull = 2, kSitePFull = 3, kSiteVhFull = 4, kSiteKvEmpty = 5,

@@ -11,7 +11,7 @@
 //               CTA loads D/2 of the D columns.
 //
 // So each SM streams only half of every K/V tile from L2 while the MMA sees
-// the full tile, without TMA multicast.
+// the full tile, and no tile is copied between the two CTAs.
 //
 // Split keys: each query row is handled by two threads (warps w and w+4 share
 // TMEM lanes 32(w%4)..+31).  Half h owns keys 64h..64h+63 of every K/V tile
@@ -26,7 +26,7 @@
 // Warps (per CTA):
 //   0-3, 4-7  softmax + epilogue (half h = warp / 4)
 //   8         TMA producers (lane 0: Q and K, lane 1: V; both CTAs load halves)
-//   9         TMEM owner; in the leader also the single MMA-issuing thread
+//   9         TMEM owner; in the leader also the MMA issuer (one elected lane)
 //   10-11     FP8 only: e4m3 -> f16 conversion of this CTA's V half
 //
 // P of half h is written over S columns 64h..64h+31 of its buffer (values
@@ -35,12 +35,14 @@
 // barriers keep every parity wait unambiguous (S(j) complete implies PV(j-2)
 // complete, and S(j+2) / PV(j+2) cannot complete before this step's P).
 #pragma once
+#include <type_traits>
+
 #include "attn_common.cuh"
 
 namespace dit {
 
-#ifndef DIT_PAIR_EXP_EMU
-#define DIT_PAIR_EXP_EMU 2
+#ifndef DIT_EXP_EMU
+#define DIT_EXP_EMU 3
 #endif
 
 template <int D_, bool FP8_>
@@ -91,8 +93,8 @@ struct PCfg {
     // Warp roles / registers.
     static constexpr int TMA_WARP = 8, MMA_WARP = 9, CONV_WARP0 = 10, CONV_THREADS = 64;
     static constexpr int THREADS = 384;
-    static constexpr int REGS_SOFTMAX = 224, REGS_OTHER = 56;   // 2 x 224 + 56 = 3 x 168
-    static constexpr int EXP_EMU = DIT_PAIR_EXP_EMU;
+    static constexpr int REGS_SOFTMAX = 192, REGS_OTHER = 120;   // 2 x 192 + 120 = 3 x 168
+    static constexpr int EXP_EMU = DIT_EXP_EMU;
     static constexpr uint32_t IDESC_QK = FP8 ? make_idesc(kFmtE4M3, kFmtE4M3, 0, 2 * kBM, kBN)
                                              : make_idesc(kFmtBF16, kFmtBF16, 0, 2 * kBM, kBN);
     static constexpr uint32_t IDESC_PV = FP8 ? make_idesc(kFmtF16, kFmtF16, 1, 2 * kBM, D)
@@ -224,77 +226,105 @@ __device__ __forceinline__ void pair_producer(const PairCtx<C> &x, const FwdPara
     }
 }
 
-// ------------------------------------------------------------------ MMA issuer (leader, one thread)
+// ------------------------------------------------------------------ MMA issuer (leader, one warp)
+// The whole warp runs the loop and one elected lane issues each MMA and
+// commit.  The issuing warp shares its SM sub-partition with two softmax
+// warps; in warp-uniform code the descriptor arithmetic stays on the uniform
+// datapath, which keeps the tensor pipe fed under that contention (a lone
+// lane-0 branch measured about 20% slower issue).  All shared-memory
+// descriptors of one operand differ only in the start-address field (bits
+// 0..13, address >> 4; addresses stay below 2^18 so the field never
+// carries), so each is a base descriptor plus a compile-time constant, and the
+// loop is unrolled over the two S buffers so that every TMEM address and
+// descriptor offset is an immediate.
 template <class C>
 __device__ __forceinline__ void pair_mma(const PairCtx<C> &x, const FwdParams &p)
 {
     auto *bars = x.bars;
     constexpr uint16_t kBoth = 0x3;
-    // S(j) into buffer j % 2 from K stage j % 2.
-    auto issue_s = [&](int buf) {
-        const uint32_t q_addr = x.base + C::OFF_Q;
-        const uint32_t k_addr = x.base + C::OFF_K + buf * align_up(C::KTILE, 1024);
-        const uint32_t tS = x.tmem + C::TM_S + 128u * buf;
+    constexpr uint32_t K_STAGE = align_up(C::KTILE, 1024);
+    constexpr uint32_t V_STAGE = C::FP8 ? align_up(C::VTILE16, 1024) : align_up(C::VRAW_TILE, 1024);
+    const uint32_t base = __shfl_sync(0xffffffffu, x.base, 0);
+    const uint32_t tmem = __shfl_sync(0xffffffffu, x.tmem, 0);
+    const uint64_t q_desc = make_smem_desc(base + C::OFF_Q, 16, 8 * C::SWZ, C::SWZ_MODE);
+    const uint64_t k_desc = make_smem_desc(base + C::OFF_K, 16, 8 * C::SWZ, C::SWZ_MODE);
+    const uint64_t v_desc =
+        make_smem_desc(base + (C::FP8 ? C::OFF_VH : C::OFF_V), 16, 8 * C::VROW, C::V_SWZ_MODE);
+    // S(j) into buffer BUF = j % 2 from K stage BUF.
+    auto issue_s = [&](auto buf_c) {
+        constexpr int BUF = decltype(buf_c)::value;
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk) {
             const uint32_t b = kk / C::STEPS_PER_BOX, w = (kk % C::STEPS_PER_BOX) * C::KSTEP;
-            const uint64_t ad = make_smem_desc(q_addr + b * C::QBOX_BYTES + w, 16, 8 * C::SWZ, C::SWZ_MODE);
-            const uint64_t bd = make_smem_desc(k_addr + b * C::KBOX_BYTES + w, 16, 8 * C::SWZ, C::SWZ_MODE);
-            if (C::FP8)
-                mma2_f8_ss(tS, ad, bd, C::IDESC_QK, kk > 0);
-            else
-                mma2_f16_ss(tS, ad, bd, C::IDESC_QK, kk > 0);
+            const uint64_t ad = q_desc + ((b * C::QBOX_BYTES + w) >> 4);
+            const uint64_t bd = k_desc + ((BUF * K_STAGE + b * C::KBOX_BYTES + w) >> 4);
+            if (elect_one()) {
+                if (C::FP8)
+                    mma2_f8_ss(tmem + C::TM_S + 128u * BUF, ad, bd, C::IDESC_QK, kk > 0);
+                else
+                    mma2_f16_ss(tmem + C::TM_S + 128u * BUF, ad, bd, C::IDESC_QK, kk > 0);
+            }
         }
     };
-    // PV(j) from buffer j % 2: key half h (P_h, V rows 64h..64h+63) into O_h.
-    auto issue_pv = [&](int buf, uint32_t v_addr, bool first) {
-        const uint32_t tS = x.tmem + C::TM_S + 128u * buf;
+    // PV(j) from buffer BUF: key half h (P_h, V rows 64h..64h+63) into O_h.
+    auto issue_pv = [&](auto buf_c, bool first) {
+        constexpr int BUF = decltype(buf_c)::value;
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
             const int h = m >> 2, kk = m & 3;
-            const uint64_t bd = make_smem_desc(v_addr + (64 * h + 16 * kk) * C::VROW, 16, 8 * C::VROW,
-                                               C::V_SWZ_MODE);
-            mma2_f16_ts(x.tmem + C::TM_O + h * C::D, tS + 64 * h + 8 * kk, bd, C::IDESC_PV,
-                        (first && kk == 0) ? 0u : 1u);
+            const uint64_t bd = v_desc + ((BUF * V_STAGE + (64 * h + 16 * kk) * C::VROW) >> 4);
+            if (elect_one())
+                mma2_f16_ts(tmem + C::TM_O + h * C::D, tmem + C::TM_S + 128u * BUF + 64 * h + 8 * kk, bd,
+                            C::IDESC_PV, (kk == 0 && first) ? 0u : 1u);
         }
-    };
-    auto v_operand = [&](int j) {
-        return C::FP8 ? x.base + C::OFF_VH + (j & 1) * align_up(C::VTILE16, 1024)
-                      : x.base + C::OFF_V + (j % 2) * align_up(C::VRAW_TILE, 1024);
     };
     bool ok = true;
-    // Everything step j needs (P(j), V(j), K(j+2)) completes one barrier.
-    auto wait_ready = [&](int j) {
-        ok = ok && wait_bar_cluster(x.bar(bars->ready[j % 2]), (j / 2) & 1, x.abort, x.lim, kSitePFull);
+    const int n = p.n_kv;
+    // Step j: once P(j), V(j) and K(j+2) are in (ready[j % 2]), PV(j) and then
+    // S(j+2) into the same buffer.  S(j+2) depends on nothing of step j+1, so
+    // the softmax of step j+1 overlaps both.
+    auto step = [&](auto buf_c, int j) {
+        constexpr int BUF = decltype(buf_c)::value;
+        ok = __all_sync(0xffffffffu,
+                        wait_bar_cluster(x.bar(bars->ready[BUF]), (j >> 1) & 1, x.abort, x.lim, kSitePFull));
+        if (!ok)
+            return;
+        tc_fence_after();
+        issue_pv(buf_c, j == 0);
+        if (elect_one())
+            mma2_commit_mc(x.bar(bars->pv_done[BUF]), kBoth);
+        if (j + 2 < n) {
+            issue_s(buf_c);
+            if (elect_one())
+                mma2_commit_mc(x.bar(bars->s_full[BUF]), kBoth);
+        }
+        __syncwarp();
     };
-    const int n = p.n_kv, n0 = n < 2 ? n : 2;
-    ok = wait_bar_cluster(x.bar(bars->q_full), 0, x.abort, x.lim, kSiteQFull) &&
-         wait_bar_cluster(x.bar(bars->k0_full), 0, x.abort, x.lim, kSiteKFull);
+    using B0 = std::integral_constant<int, 0>;
+    using B1 = std::integral_constant<int, 1>;
+    ok = __all_sync(0xffffffffu, wait_bar_cluster(x.bar(bars->q_full), 0, x.abort, x.lim, kSiteQFull) &&
+                                     wait_bar_cluster(x.bar(bars->k0_full), 0, x.abort, x.lim, kSiteKFull));
     if (ok) {
         tc_fence_after();
-        for (int s = 0; s < n0; ++s) {
-            issue_s(s);
-            mma2_commit_mc(x.bar(bars->s_full[s]), kBoth);
+        issue_s(B0{});
+        if (elect_one())
+            mma2_commit_mc(x.bar(bars->s_full[0]), kBoth);
+        if (n > 1) {
+            issue_s(B1{});
+            if (elect_one())
+                mma2_commit_mc(x.bar(bars->s_full[1]), kBoth);
         }
+        __syncwarp();
     }
-    // Per step j: once P(j), V(j) and K(j+2) are in (ready[j % 2]), PV(j) and
-    // then S(j+2) into the same buffer.  S(j+2) depends on nothing of step
-    // j+1, so the softmax of step j+1 overlaps both.
-    for (int j = 0; j < n; ++j) {
-        const int buf = j % 2;
-        wait_ready(j);
-        if (!ok)
-            break;
-        tc_fence_after();
-        issue_pv(buf, v_operand(j), j == 0);
-        mma2_commit_mc(x.bar(bars->pv_done[buf]), kBoth);
-        if (j + 2 < n) {
-            issue_s(buf);
-            mma2_commit_mc(x.bar(bars->s_full[buf]), kBoth);
-        }
+    for (int j = 0; j < n && ok; j += 2) {
+        step(B0{}, j);
+        if (j + 1 < n && ok)
+            step(B1{}, j + 1);
     }
     if (!ok) {
-        mma2_commit(x.bar(bars->drain));
+        if (elect_one())
+            mma2_commit(x.bar(bars->drain));
+        __syncwarp();
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(x.bar(bars->drain), 0) && globaltimer_ns() - t0 < 50000000ull) {
         }
@@ -374,6 +404,9 @@ __device__ __forceinline__ float half_row_max(const uint32_t (&s)[2][32], int kb
 // p = 2^(s*c2 - mc) for this thread's 64 values, packed to 16 bits and stored
 // as 32 TMEM columns at tS (over S values only this thread has read).
 // Returns the sum of the p.  Of every 8 pairs, EMU use the FMA-pipe exp2.
+// bf16 P takes the high halves of the two f32 (one byte permute: truncation,
+// made unbiased by the kTruncGain factor the caller folds into mc); f16 P
+// (FP8 path) is rounded to nearest.
 template <class C, bool MASK, int EMU>
 __device__ __forceinline__ float half_row_exp_store(const uint32_t (&s)[2][32], uint32_t tS, int kbase, int valid,
                                                     float c2, float mc)
@@ -401,7 +434,8 @@ __device__ __forceinline__ float half_row_exp_store(const uint32_t (&s)[2][32], 
                 e.y = (kbase + 32 * i + c + 1 < valid) ? e.y : 0.f;
             }
             acc[pi & 3] = __fadd2_rn(acc[pi & 3], e);
-            pk[c / 2] = pack_p(e.x, e.y, C::FP8);
+            pk[c / 2] = C::FP8 ? pack_p(e.x, e.y, true)
+                               : __byte_perm(__float_as_uint(e.x), __float_as_uint(e.y), 0x7632);
         }
         tmem_st16(tS + 16 * i, pk);
     }
@@ -447,7 +481,8 @@ __device__ __forceinline__ void half_row_step(const PairCtx<C> &x, const FwdPara
         alpha = ex2_approx((st.m_use - mx) * st.c2);
         st.m_use = mx;
     }
-    const float mc = st.m_use * st.c2;
+    // bf16 P is truncated; kTruncLog2 makes it unbiased (attn_common.cuh).
+    const float mc = st.m_use * st.c2 - (C::FP8 ? 0.f : kTruncLog2);
     const float sum = masked ? half_row_exp_store<C, true, C::EXP_EMU>(s, tS, 64 * h, p.kv_tail, st.c2, mc)
                              : half_row_exp_store<C, false, C::EXP_EMU>(s, tS, 64 * h, kBN, st.c2, mc);
     st.l = st.l * alpha + sum;
@@ -527,7 +562,7 @@ __device__ __forceinline__ void pair_softmax(const PairCtx<C> &x, const FwdParam
     const uint32_t ost = C::FP8 ? x.base + C::OFF_OST : x.base + C::OFF_Q;
     if (alive) {
         tc_fence_after();
-        const float inv = vs / l_row;
+        const float inv = (C::FP8 ? vs : kTruncGain) / l_row;
         const float w0 = a0 * inv, w1 = a1 * inv;
         // This thread writes output columns h*D/2 .. h*D/2 + D/2 of its row.
         const uint32_t tO0 = x.tmem + lane_off + C::TM_O + h * (D / 2);
@@ -559,7 +594,7 @@ __device__ __forceinline__ void pair_softmax(const PairCtx<C> &x, const FwdParam
     if (alive) {
         const int qrow = x.q0 + row;
         if (h == 0 && p.lse != nullptr && qrow < p.L)
-            p.lse[(long long)x.bh * p.L + qrow] = (mrow + log2f(l_row)) * kLn2;
+            p.lse[(long long)x.bh * p.L + qrow] = (mrow + log2f(l_row) - (C::FP8 ? 0.f : kTruncLog2)) * kLn2;
         if (warp == 0 && lane == 0) {
             for (int b = 0; b < C::OBOX; ++b)
                 tma_store_3d(tm_o, ost + b * C::OBOX_BYTES, b * 64, x.q0, x.bh);
@@ -631,7 +666,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (lane < 2)
                 pair_producer<C>(x, p, lane, &tm_q, &tm_k, &tm_v);
         } else if (warp == C::MMA_WARP) {
-            if (lane == 0 && rank == 0)
+            if (rank == 0)
                 pair_mma<C>(x, p);
         } else if (FP8) {
             pair_convert_v<C>(x, p);

@@ -280,6 +280,15 @@ __device__ __forceinline__ uint32_t cluster_ctarank()
 }
 
 // Shared-memory address of the same variable in CTA `rank` of the cluster.
+// One lane of a converged warp (the same lane in every lane's view).
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred = 0;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(pred));
+    return pred != 0;
+}
+
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
 {
     uint32_t r;
