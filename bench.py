@@ -58,7 +58,10 @@ def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "attention_dit_attn_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
+        path = os.path.join(csrc, name)
+        if not (os.path.isfile(path) and name.endswith((".cu", ".cuh", ".h", ".py"))):
+            continue
+        with open(path, "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
