@@ -8,6 +8,7 @@ if the library is missing or cannot run, calls raise.
     import attention_dit_attn_b200 as dit
     o, lse = dit.dit_attn_fwd(q, k, v)                    # bf16 [B,H,L,D] on cuda
     o, lse = dit.dit_attn_fwd(q8, k8, v8, q_scale=qs, k_scale=ks, v_scale=vs)  # e4m3
+    o, lse = dit.dit_attn_lse_merge([(o0, lse0), (o1, lse1)])   # combine key chunks
 """
 from __future__ import annotations
 
@@ -21,12 +22,14 @@ from . import _build
 __all__ = [
     "DIT_ATTN_BF16", "DIT_ATTN_FP8_E4M3", "DitAttnError", "dit_attn_fwd", "dit_attn_fwd_ptr",
     "dit_attn_status_string", "dit_attn_check_device_error", "dit_attn_set_wait_limit_ns",
-    "dit_attn_selftest_wait_timeout", "dit_attn_launches_per_call", "ensure_built", "lib",
-    "header_functions", "STATUS",
+    "dit_attn_selftest_wait_timeout", "dit_attn_launches_per_call", "dit_attn_lse_merge",
+    "dit_attn_lse_merge_ptr", "DIT_ATTN_MERGE_MAX_PARTS", "ensure_built", "lib", "header_functions",
+    "STATUS",
 ]
 
 DIT_ATTN_BF16 = 0
 DIT_ATTN_FP8_E4M3 = 1
+DIT_ATTN_MERGE_MAX_PARTS = 8
 
 STATUS = {
     0: "DIT_ATTN_OK", 1: "DIT_ATTN_ERR_NULL", 2: "DIT_ATTN_ERR_SHAPE", 3: "DIT_ATTN_ERR_DTYPE",
@@ -71,6 +74,9 @@ def lib() -> ctypes.CDLL:
         L.dit_attn_selftest_wait_timeout.argtypes = [u64, vp]
         L.dit_attn_launches_per_call.restype = i32
         L.dit_attn_launches_per_call.argtypes = [i32, i32, i32, i32, i32]
+        L.dit_attn_lse_merge.restype = i32
+        L.dit_attn_lse_merge.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i32, vp, vp,
+                                         ctypes.c_longlong, i32, vp]
         _lib = L
     return _lib
 
@@ -168,3 +174,51 @@ def dit_attn_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
 
 def dit_attn_launches_per_call(B: int, H: int, L: int, D: int, dtype: int) -> int:
     return lib().dit_attn_launches_per_call(B, H, L, D, dtype)
+
+
+def dit_attn_lse_merge_ptr(o_parts: list[int], lse_parts: list[int], o: int, lse: int | None,
+                           rows: int, D: int, stream: int = 0) -> int:
+    """Raw C-ABI call with integer device pointers; returns the status code."""
+    n = len(o_parts)
+    if n != len(lse_parts):
+        raise ValueError("one lse pointer per partial output")
+    op = (ctypes.c_void_p * max(n, 1))(*o_parts)
+    lp = (ctypes.c_void_p * max(n, 1))(*lse_parts)
+    return lib().dit_attn_lse_merge(op, lp, n, o, lse, rows, D, stream)
+
+
+def dit_attn_lse_merge(parts, o=None, lse=None, *, want_lse: bool = True, stream=None):
+    """Merge partial attention results over disjoint key chunks.
+
+    parts: sequence of (o_c, lse_c) pairs as returned by dit_attn_fwd for the same
+    query rows: o_c bf16 [..., D] and lse_c fp32 [...] on CUDA, all of one shape.
+    Allocates o and lse when not given (either may be parts[0]'s own tensors, for
+    an in-place merge).  Asynchronous on ``stream``.  Returns (o, lse)."""
+    import torch
+    if not 1 <= len(parts) <= DIT_ATTN_MERGE_MAX_PARTS:
+        raise ValueError(f"between 1 and {DIT_ATTN_MERGE_MAX_PARTS} parts")
+    o0, l0 = parts[0]
+    shape, D = tuple(o0.shape), o0.shape[-1]
+    rows = o0.numel() // D
+    for oc, lc in parts:
+        if not (isinstance(oc, torch.Tensor) and oc.is_cuda and oc.dtype == torch.bfloat16
+                and oc.is_contiguous() and tuple(oc.shape) == shape):
+            raise ValueError("every partial o must be a contiguous bf16 CUDA tensor of one shape")
+        if not (isinstance(lc, torch.Tensor) and lc.is_cuda and lc.dtype == torch.float32
+                and lc.is_contiguous() and lc.numel() == rows):
+            raise ValueError("every partial lse must be a contiguous fp32 CUDA tensor with one value per row")
+    if o is None:
+        o = torch.empty(shape, dtype=torch.bfloat16, device=o0.device)
+    elif tuple(o.shape) != shape or o.dtype != torch.bfloat16 or not o.is_contiguous() or not o.is_cuda:
+        raise ValueError("o must be a contiguous bf16 CUDA tensor shaped like the parts")
+    if lse is None and want_lse:
+        lse = torch.empty(tuple(l0.shape), dtype=torch.float32, device=o0.device)
+    elif lse is not None and (lse.numel() != rows or lse.dtype != torch.float32
+                              or not lse.is_contiguous() or not lse.is_cuda):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor with one value per row")
+    rc = dit_attn_lse_merge_ptr([oc.data_ptr() for oc, _ in parts], [lc.data_ptr() for _, lc in parts],
+                                o.data_ptr(), None if lse is None else lse.data_ptr(), rows, D,
+                                _stream_handle(stream))
+    if rc != 0:
+        raise DitAttnError(rc, "dit_attn_lse_merge: ")
+    return o, lse

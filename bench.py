@@ -16,6 +16,11 @@ hot path is one kernel launch).  Prints ONE JSON line on rank 0.
   the workload's query rows (rank 0, N=1 only).
 * --impl reference: the oracle alone, as the reference arm, on the same
   workload and metric.
+* --op lse_merge: instead of the forward, the LSE merge of --parts partial
+  attentions (ring attention's combine step) over the workload's rows; the
+  parts are real partial results (each query chunk against each key chunk,
+  computed once before timing).  Metric: GB/s of algorithmic HBM traffic,
+  roofline against the measured copy bandwidth.
 Multi-GPU (torchrun): every rank runs its own replica (no data exchange:
 heads and batches are independent), scaling "weak".
 """
@@ -36,6 +41,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attention TFLOP/s and % of B200 tensor-core peak at 1 GPU"
+MERGE_METRIC = "LSE merge of partial attentions: GB/s of algorithmic HBM traffic at 1 GPU"
 DEFAULT_WORKLOAD = "flux_2048_cfg"      # the first workload with L >= 16k (the stated target)
 NOMINAL_TFLOPS = {"bf16": 2250.0, "e4m3": 4500.0}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
@@ -66,10 +72,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, kind: str = "attn_fwd"):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source (its source hash matches); else None."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{kind}_{workload}.md")
     try:
         text = open(path).read()
     except OSError:
@@ -281,6 +287,195 @@ def workload_config(w):
             "parallelism": "replicas"}
 
 
+# ------------------------------------------------------------------ LSE merge (ring-attention combine)
+
+def merge_bytes(rows: int, D: int, n: int) -> int:
+    """Algorithmic bytes of one merge: n parts of bf16 o + fp32 lse read, one written."""
+    return rows * (n * (2 * D + 4) + 2 * D + 4)
+
+
+def make_merge_parts(w, inp, dev, n: int):
+    """Ring degree n over the workload's sequence: part c holds, for every query
+    chunk r, dit_attn_fwd(Q_r, K_c, V_c); rows ordered (r, b, h, l)."""
+    import torch
+    import attention_dit_attn_b200 as dit
+    if w.L % n:
+        raise ValueError(f"L={w.L} does not split into {n} equal chunks")
+    Lc = w.L // n
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    kw = {}
+    if inp.q_scale is not None:
+        kw = dict(q_scale=inp.q_scale.to(dev).contiguous(), k_scale=inp.k_scale.to(dev).contiguous(),
+                  v_scale=inp.v_scale.to(dev).contiguous())
+    chunk = lambda t, i: t[:, :, i * Lc:(i + 1) * Lc].contiguous()
+    parts = []
+    for c in range(n):
+        outs = [dit.dit_attn_fwd(chunk(q, r), chunk(k, c), chunk(v, c), scale=w.scale, **kw) for r in range(n)]
+        parts.append((torch.stack([o for o, _ in outs]).reshape(-1, w.D).contiguous(),
+                      torch.stack([l for _, l in outs]).reshape(-1).contiguous()))
+    torch.cuda.synchronize(dev)
+    return parts
+
+
+def merge_oracle_rate(parts_cpu, seconds: float):
+    """The fp64 merge oracle on a bounded sample of rows: (GB/s algorithmic, rows, s)."""
+    from oracle.lse_merge import lse_merge
+    rows_total, D = parts_cpu[0][0].shape
+    n = len(parts_cpu)
+    rows = min(rows_total, 4096)
+    while True:
+        t0 = time.perf_counter()
+        lse_merge([o[:rows].double().numpy() for o, _ in parts_cpu], [l[:rows].double().numpy() for _, l in parts_cpu])
+        dt = time.perf_counter() - t0
+        if dt >= seconds / 4 or rows >= rows_total:
+            break
+        rows = min(rows_total, rows * 4)
+    return merge_bytes(rows, D, n) / dt / 1e9, rows, dt
+
+
+def merge_config(w, n, rows):
+    return {"workload": w.name, "op": "lse_merge", "parts": n, "rows": rows, "D": w.D,
+            "B": w.B, "H": w.H, "L": w.L, "ring_degree": n, "input_dtype": "bf16 o + fp32 lse",
+            "output_dtype": "bf16 o + fp32 lse", "bytes_per_call": merge_bytes(rows, w.D, n),
+            "l2": "inputs larger than L2" if merge_bytes(rows, w.D, n) > L2_BYTES
+            else "L2 flushed between timed steps (256 MB write)",
+            "parallelism": "replicas"}
+
+
+def run_merge_reference(args, dist: Dist):
+    if dist.rank != 0:
+        return
+    import torch
+    from attention_dit_attn_b200 import workloads as wl
+    w = wl.ALL[args.workload]
+    n = args.parts
+    rows = w.B * w.H * w.L
+    g = torch.Generator().manual_seed(w.seed)
+    sample = min(rows, 1 << 16)
+    parts = [(torch.randn((sample, w.D), generator=g).to(torch.bfloat16), torch.randn((sample,), generator=g))
+             for _ in range(n)]
+    per = 60.0 / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        merge_oracle_rate(parts, per)
+    rates = [merge_oracle_rate(parts, per) for _ in range(args.steps)]
+    value = statistics.median(r[0] for r in rates)
+    cores = 1
+    line = {
+        "impl": "reference", "metric": MERGE_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * merge_bytes(rows, w.D, n) / (value * 1e9),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": merge_config(w, n, rows),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: fp64 numpy merge oracle on {rates[0][1]} rows of {n} parts"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_merge(args, dist: Dist):
+    import torch
+    import attention_dit_attn_b200 as dit
+    from attention_dit_attn_b200 import workloads as wl
+
+    dit.ensure_built()
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    w = wl.ALL[args.workload]
+    n = args.parts
+    parts = make_merge_parts(w, wl.generate_workload(w), dev, n)
+    rows = parts[0][0].shape[0]
+    nbytes = merge_bytes(rows, w.D, n)
+    o = torch.empty_like(parts[0][0])
+    lse = torch.empty_like(parts[0][1])
+    flush = None
+    if nbytes <= L2_BYTES:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        dit.dit_attn_lse_merge(parts, o, lse, stream=stream)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler()
+    if dist.rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in evs:
+        if flush is not None:
+            flush.fill_(1)
+        a.record(stream)
+        dit.dit_attn_lse_merge(parts, o, lse, stream=stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    seconds = sum(a.elapsed_time(b) for a, b in evs) / 1e3
+    dist.barrier()
+    if dist.rank == 0:
+        time.sleep(0.2)
+        sampler.stop()
+    max_seconds = dist.max(seconds, dev)
+    value = nbytes * args.steps * dist.world / max_seconds / 1e9
+    achieved = nbytes / (seconds / args.steps) / 1e9
+
+    # end to end: parts from pinned host memory, merged result back to the host
+    e2e_steps = max(3, min(args.steps, 10))
+    hparts = [(po.cpu().pin_memory(), pl.cpu().pin_memory()) for po, pl in parts]
+    dparts = [(torch.empty_like(po), torch.empty_like(pl)) for po, pl in parts]
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_step():
+        for (ho_, hl_), (do_, dl_) in zip(hparts, dparts):
+            do_.copy_(ho_, non_blocking=True)
+            dl_.copy_(hl_, non_blocking=True)
+        dit.dit_attn_lse_merge(dparts, o, lse, stream=stream)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = dist.max(a.elapsed_time(b) / 1e3, dev)
+    h2d = sum(po.numel() * 2 + pl.numel() * 4 for po, pl in hparts)
+    d2h = ho.numel() * 2 + hl.numel() * 4
+
+    peaks, peaks_kind = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    traffic = profiled_traffic(w.name, kind="lse_merge")
+    clocks = sampler.summary(physical_gpu_index(dist.local_rank)) if dist.rank == 0 else {}
+    line = {
+        "metric": MERGE_METRIC, "value": value, "unit": "GB/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * max_seconds / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": merge_config(w, n, rows),
+        "e2e": {"value": nbytes * e2e_steps * dist.world / e2e_s / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "result_matches_device": torch.equal(ho, o.cpu())},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"HBM copy, {peaks_kind}", "traffic": traffic,
+                     "kernel": "lse_merge_kernel", "bytes_per_launch": nbytes},
+        "clocks": clocks,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        parts_cpu = [(po[: 1 << 16].cpu(), pl[: 1 << 16].cpu()) for po, pl in parts]
+        rate, srows, dt = merge_oracle_rate(parts_cpu, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": f"fp64 numpy merge oracle on the first {srows} rows of the "
+                                          f"{n} parts: {dt:.2f} s"}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, dist: Dist):
     import torch
     import attention_dit_attn_b200 as dit
@@ -430,20 +625,24 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["attention", "lse_merge"], default="attention")
+    ap.add_argument("--parts", type=int, default=2, help="lse_merge: number of partial results (ring degree)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from attention_dit_attn_b200 import workloads as wl
     if args.workload not in wl.ALL:
         ap.error(f"--workload must be one of {list(wl.ALL)}")
+    if not 1 <= args.parts <= 8:
+        ap.error("--parts must be 1..8")
     if args.impl == "reference":
         # The oracle runs on rank 0's host cores only; other ranks exit at once.
         if int(os.environ.get("RANK", "0")) == 0:
-            run_reference(args, Dist.single())
+            (run_merge_reference if args.op == "lse_merge" else run_reference)(args, Dist.single())
         return
     dist = Dist(args.gpus)
     try:
-        run_ours(args, dist)
+        (run_merge if args.op == "lse_merge" else run_ours)(args, dist)
     finally:
         dist.close()
 

@@ -121,6 +121,51 @@ int dit_attn_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
  */
 int dit_attn_launches_per_call(int B, int H, int L, int D, int dtype);
 
+/* Largest number of partial results dit_attn_lse_merge combines in one call. */
+#define DIT_ATTN_MERGE_MAX_PARTS 8
+
+/*
+ * dit_attn_lse_merge — combines partial attention results over disjoint key
+ * chunks into the result over their union, asynchronous on `stream`.
+ *
+ * This is the combine step of ring attention / USP: a block of query rows
+ * meets the K/V chunks one at a time and the partial results are merged.
+ * The xDiT paper cites both methods in its reference list ("xDiT: an
+ * Inference Engine for Diffusion Transformers (DiTs) with Massive
+ * Parallelism"), and the 2-GPU script of the page "Accelerating Diffusers and
+ * xDiT Image Generation with MXFP4 using AMD Quark on AMD Instinct MI350 GPUs"
+ * sets its `ring degree`.  The pages give no formula; the exact log-sum-exp
+ * rule is used.  Per row,
+ *
+ *     lse = M + log sum_c exp(lse_c - M),   M = max_c lse_c,
+ *     o   = sum_c exp(lse_c - lse) o_c,
+ *
+ * and a row whose parts all have lse = -inf gives o = 0, lse = -inf.  The
+ * (o_c, lse_c) are exactly what dit_attn_fwd returns for the same query rows
+ * over key chunk c.
+ *
+ * o_parts   host array of n_parts device pointers, each to [rows, D] bf16
+ *           (e.g. [B, H, L, D] with rows = B*H*L); 16-byte aligned.
+ * lse_parts host array of n_parts device pointers, each to [rows] fp32
+ *           natural-log LSE (-inf allowed: an empty chunk); 4-byte aligned.
+ * n_parts   1 .. DIT_ATTN_MERGE_MAX_PARTS.
+ * o         device pointer to [rows, D] bf16, 16-byte aligned; may be the
+ *           same buffer as any o_parts[c] (each element is read before it is
+ *           written, by the same thread).
+ * lse       device pointer to [rows] fp32, or NULL to skip it; may be the
+ *           same buffer as any lse_parts[c].
+ * rows      >= 0; rows * D < 2^40.  With rows = 0 nothing is enqueued and
+ *           the device pointers are not examined (they may be NULL).
+ * D         64 or 128.
+ *
+ * Ownership: the caller owns every buffer; the host arrays are read during
+ * the call only.  Errors: argument errors (DIT_ATTN_ERR_NULL, _SHAPE,
+ * _ALIGN, _ARCH) are reported before anything is enqueued; a launch failure
+ * returns DIT_ATTN_ERR_LAUNCH.  The kernel has no waits.
+ */
+int dit_attn_lse_merge(const void *const *o_parts, const float *const *lse_parts, int n_parts,
+                       void *o, float *lse, long long rows, int D, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

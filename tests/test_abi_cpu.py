@@ -18,7 +18,7 @@ def test_library_exports_every_header_function(L):
     names = dit.header_functions()
     assert set(names) == {"dit_attn_fwd", "dit_attn_status_string", "dit_attn_check_device_error",
                           "dit_attn_set_wait_limit_ns", "dit_attn_selftest_wait_timeout",
-                          "dit_attn_launches_per_call"}
+                          "dit_attn_launches_per_call", "dit_attn_lse_merge"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -69,3 +69,28 @@ def test_python_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         dit.dit_attn_fwd(x, x, x)
+
+
+@pytest.mark.parametrize("o_parts,lse_parts,o,rows,D,want", [
+    ([0], [16], 16, 4, 128, 1),                 # a part's o NULL
+    ([16], [0], 16, 4, 128, 1),                 # a part's lse NULL
+    ([16], [16], 0, 4, 128, 1),                 # output NULL
+    ([], [], 16, 4, 128, 2),                    # no parts
+    ([16] * 9, [16] * 9, 16, 4, 128, 2),        # more than DIT_ATTN_MERGE_MAX_PARTS
+    ([16], [16], 16, 4, 96, 2),                 # D not 64 / 128
+    ([16], [16], 16, -1, 128, 2),               # negative rows
+    ([16], [16], 16, 1 << 34, 128, 2),          # rows * D >= 2^40
+    ([24], [16], 16, 4, 128, 4),                # part o not 16-byte aligned
+    ([16], [18], 16, 4, 128, 4),                # part lse not 4-byte aligned
+    ([16], [16], 8, 4, 128, 4),                 # output not 16-byte aligned
+])
+def test_lse_merge_argument_validation(L, o_parts, lse_parts, o, rows, D, want):
+    assert dit.dit_attn_lse_merge_ptr(o_parts, lse_parts, o, None, rows, D) == want
+
+
+def test_lse_merge_wellformed_call_without_gpu_reports_arch(L):
+    assert dit.dit_attn_lse_merge_ptr([16, 32], [16, 32], 16, 64, 10, 64) == 5
+
+
+def test_lse_merge_zero_rows_is_a_no_op_even_with_null_buffers(L):
+    assert dit.dit_attn_lse_merge_ptr([0, 0], [0, 0], 0, None, 0, 128) == 0
