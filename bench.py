@@ -60,14 +60,18 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+# Source files of each kernel: a committed ncu summary is used only while these match.
+KERNEL_SOURCES = {
+    "attn_fwd": ["attn_common.cuh", "attn_fwd_sm100.cuh", "dit_attn.cu", "exp2_poly_fit.py", "sm100_ptx.cuh"],
+    "lse_merge": ["lse_merge.cu"],
+}
+
+
+def kernel_source_hash(kind: str = "attn_fwd") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "attention_dit_attn_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        path = os.path.join(csrc, name)
-        if not (os.path.isfile(path) and name.endswith((".cu", ".cuh", ".h", ".py"))):
-            continue
-        with open(path, "rb") as f:
+    for name in sorted(KERNEL_SOURCES[kind]):
+        with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
@@ -82,7 +86,7 @@ def profiled_traffic(workload: str, kind: str = "attn_fwd"):
         return None
     m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
     m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash(kind):
         return None
     return float(m_bytes.group(1))
 
