@@ -9,6 +9,7 @@ if the library is missing or cannot run, calls raise.
     o, lse = dit.dit_attn_fwd(q, k, v)                    # bf16 [B,H,L,D] on cuda
     o, lse = dit.dit_attn_fwd(q8, k8, v8, q_scale=qs, k_scale=ks, v_scale=vs)  # e4m3
     o, lse = dit.dit_attn_lse_merge([(o0, lse0), (o1, lse1)])   # combine key chunks
+    diff, reuse = dit.dit_attn_residual_diff(r_now, r_prev, 0.12)  # step-cache decision
 """
 from __future__ import annotations
 
@@ -23,8 +24,9 @@ __all__ = [
     "DIT_ATTN_BF16", "DIT_ATTN_FP8_E4M3", "DitAttnError", "dit_attn_fwd", "dit_attn_fwd_ptr",
     "dit_attn_status_string", "dit_attn_check_device_error", "dit_attn_set_wait_limit_ns",
     "dit_attn_selftest_wait_timeout", "dit_attn_launches_per_call", "dit_attn_lse_merge",
-    "dit_attn_lse_merge_ptr", "DIT_ATTN_MERGE_MAX_PARTS", "ensure_built", "lib", "header_functions",
-    "STATUS",
+    "dit_attn_lse_merge_ptr", "DIT_ATTN_MERGE_MAX_PARTS", "dit_attn_residual_diff",
+    "dit_attn_residual_diff_ptr", "dit_attn_residual_diff_workspace_bytes", "ensure_built", "lib",
+    "header_functions", "STATUS",
 ]
 
 DIT_ATTN_BF16 = 0
@@ -74,6 +76,11 @@ def lib() -> ctypes.CDLL:
         L.dit_attn_selftest_wait_timeout.argtypes = [u64, vp]
         L.dit_attn_launches_per_call.restype = i32
         L.dit_attn_launches_per_call.argtypes = [i32, i32, i32, i32, i32]
+        L.dit_attn_residual_diff_workspace_bytes.restype = ctypes.c_size_t
+        L.dit_attn_residual_diff_workspace_bytes.argtypes = [ctypes.c_longlong]
+        L.dit_attn_residual_diff.restype = i32
+        L.dit_attn_residual_diff.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_float, vp, ctypes.c_size_t,
+                                             vp, vp, vp]
         L.dit_attn_lse_merge.restype = i32
         L.dit_attn_lse_merge.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i32, vp, vp,
                                          ctypes.c_longlong, i32, vp]
@@ -222,3 +229,46 @@ def dit_attn_lse_merge(parts, o=None, lse=None, *, want_lse: bool = True, stream
     if rc != 0:
         raise DitAttnError(rc, "dit_attn_lse_merge: ")
     return o, lse
+
+
+def dit_attn_residual_diff_workspace_bytes(n: int) -> int:
+    return int(lib().dit_attn_residual_diff_workspace_bytes(int(n)))
+
+
+def dit_attn_residual_diff_ptr(cur: int, prev: int, n: int, threshold: float, workspace: int,
+                               workspace_bytes: int, diff_out: int | None, reuse_out: int | None,
+                               stream: int = 0) -> int:
+    """Raw C-ABI call with integer device pointers; returns the status code."""
+    return lib().dit_attn_residual_diff(cur, prev, n, ctypes.c_float(threshold), workspace, workspace_bytes,
+                                        diff_out, reuse_out, stream)
+
+
+def dit_attn_residual_diff(cur, prev, threshold: float = 0.12, *, workspace=None, diff=None, reuse=None,
+                           stream=None):
+    """Step-cache decision on two bf16 CUDA tensors of equal size (the first blocks'
+    residual now and at the previous step): relative L1 change and reuse flag, as
+    one-element fp32 / int32 CUDA tensors (not synchronised).  ``workspace`` (a zeroed
+    uint8 CUDA tensor of dit_attn_residual_diff_workspace_bytes(n) bytes) may be kept
+    and passed again; it is allocated zeroed when not given."""
+    import torch
+    for name, t in (("cur", cur), ("prev", prev)):
+        if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if cur.numel() != prev.numel():
+        raise ValueError("cur and prev must have the same number of elements")
+    n = cur.numel()
+    need = dit_attn_residual_diff_workspace_bytes(n)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=cur.device)
+    elif not (workspace.is_cuda and workspace.dtype == torch.uint8 and workspace.is_contiguous()
+              and workspace.numel() >= need):
+        raise ValueError(f"workspace must be a contiguous uint8 CUDA tensor of at least {need} bytes")
+    if diff is None:
+        diff = torch.empty(1, dtype=torch.float32, device=cur.device)
+    if reuse is None:
+        reuse = torch.empty(1, dtype=torch.int32, device=cur.device)
+    rc = dit_attn_residual_diff_ptr(cur.data_ptr(), prev.data_ptr(), n, float(threshold), workspace.data_ptr(),
+                                    workspace.numel(), diff.data_ptr(), reuse.data_ptr(), _stream_handle(stream))
+    if rc != 0:
+        raise DitAttnError(rc, "dit_attn_residual_diff: ")
+    return diff, reuse

@@ -21,6 +21,9 @@ hot path is one kernel launch).  Prints ONE JSON line on rank 0.
   parts are real partial results (each query chunk against each key chunk,
   computed once before timing).  Metric: GB/s of algorithmic HBM traffic,
   roofline against the measured copy bandwidth.
+* --op residual_diff: the step-cache reuse decision (relative L1 change of a
+  hidden-state-sized bf16 residual, B*L*H*D elements of the workload, against
+  the previous step's); GB/s of algorithmic HBM traffic.
 Multi-GPU (torchrun): every rank runs its own replica (no data exchange:
 heads and batches are independent), scaling "weak".
 """
@@ -42,6 +45,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "attention TFLOP/s and % of B200 tensor-core peak at 1 GPU"
 MERGE_METRIC = "LSE merge of partial attentions: GB/s of algorithmic HBM traffic at 1 GPU"
+DIFF_METRIC = "step-cache residual-change decision: GB/s of algorithmic HBM traffic at 1 GPU"
 DEFAULT_WORKLOAD = "flux_2048_cfg"      # the first workload with L >= 16k (the stated target)
 NOMINAL_TFLOPS = {"bf16": 2250.0, "e4m3": 4500.0}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
@@ -64,6 +68,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "attn_fwd": ["attn_common.cuh", "attn_fwd_sm100.cuh", "dit_attn.cu", "exp2_poly_fit.py", "sm100_ptx.cuh"],
     "lse_merge": ["lse_merge.cu"],
+    "residual_diff": ["residual_diff.cu"],
 }
 
 
@@ -480,6 +485,168 @@ def run_merge(args, dist: Dist):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ step-cache decision (DBCache)
+
+def diff_inputs(w, dev):
+    """Seeded residuals of the workload's hidden-state size: prev ~ N(0,1), cur = prev
+    + 0.05 N(0,1) (a step whose work is reused at the published threshold 0.12)."""
+    import torch
+    n = w.B * w.L * w.H * w.D
+    g = torch.Generator(device=dev).manual_seed(w.seed)
+    prev = torch.randn(n, generator=g, device=dev)
+    cur = (prev + 0.05 * torch.randn(n, generator=g, device=dev)).to(torch.bfloat16)
+    return cur, prev.to(torch.bfloat16)
+
+
+def diff_config(w, n):
+    return {"workload": w.name, "op": "residual_diff", "elements": n, "B": w.B, "L": w.L,
+            "hidden": w.H * w.D, "input_dtype": "bf16", "threshold": 0.12, "bytes_per_call": 4 * n + 8,
+            "l2": "inputs larger than L2" if 4 * n > L2_BYTES else "L2 flushed between timed steps (256 MB write)",
+            "parallelism": "replicas"}
+
+
+def diff_oracle_rate(cur_cpu, prev_cpu, seconds: float):
+    from oracle.residual_diff import residual_diff
+    n = min(cur_cpu.numel(), 1 << 20)
+    while True:
+        c, pv = cur_cpu[:n].double().numpy(), prev_cpu[:n].double().numpy()
+        t0 = time.perf_counter()
+        residual_diff(c, pv)
+        dt = time.perf_counter() - t0
+        if dt >= seconds / 4 or n >= cur_cpu.numel():
+            return 4 * n / dt / 1e9, n, dt
+        n = min(cur_cpu.numel(), n * 4)
+
+
+def run_diff_reference(args, dist: Dist):
+    if dist.rank != 0:
+        return
+    import torch
+    from attention_dit_attn_b200 import workloads as wl
+    w = wl.ALL[args.workload]
+    n = w.B * w.L * w.H * w.D
+    g = torch.Generator().manual_seed(w.seed)
+    m = min(n, 1 << 24)
+    prev = torch.randn(m, generator=g)
+    cur = (prev + 0.05 * torch.randn(m, generator=g)).to(torch.bfloat16)
+    prev = prev.to(torch.bfloat16)
+    per = 60.0 / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        diff_oracle_rate(cur, prev, per)
+    rates = [diff_oracle_rate(cur, prev, per) for _ in range(args.steps)]
+    value = statistics.median(r[0] for r in rates)
+    line = {
+        "impl": "reference", "metric": DIFF_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * 4 * n / (value * 1e9),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": diff_config(w, n),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: fp64 numpy oracle on {rates[0][1]} elements"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_diff(args, dist: Dist):
+    import torch
+    import attention_dit_attn_b200 as dit
+    from attention_dit_attn_b200 import workloads as wl
+
+    dit.ensure_built()
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    w = wl.ALL[args.workload]
+    cur, prev = diff_inputs(w, dev)
+    n = cur.numel()
+    nbytes = 4 * n + 8
+    ws = torch.zeros(dit.dit_attn_residual_diff_workspace_bytes(n), dtype=torch.uint8, device=dev)
+    d = torch.empty(1, dtype=torch.float32, device=dev)
+    r = torch.empty(1, dtype=torch.int32, device=dev)
+    flush = None
+    if 4 * n <= L2_BYTES:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda c, p: dit.dit_attn_residual_diff(c, p, 0.12, workspace=ws, diff=d, reuse=r, stream=stream)
+    for _ in range(args.warmup):
+        call(cur, prev)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler()
+    if dist.rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in evs:
+        if flush is not None:
+            flush.fill_(1)
+        a.record(stream)
+        call(cur, prev)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    seconds = sum(a.elapsed_time(b) for a, b in evs) / 1e3
+    dist.barrier()
+    if dist.rank == 0:
+        time.sleep(0.2)
+        sampler.stop()
+    max_seconds = dist.max(seconds, dev)
+    value = nbytes * args.steps * dist.world / max_seconds / 1e9
+    achieved = nbytes / (seconds / args.steps) / 1e9
+
+    # end to end: both residuals from pinned host memory, the decision back to the host
+    e2e_steps = max(3, min(args.steps, 10))
+    hc, hp = cur.cpu().pin_memory(), prev.cpu().pin_memory()
+    dc, dp = torch.empty_like(cur), torch.empty_like(prev)
+    hd = torch.empty(1, dtype=torch.float32).pin_memory()
+    hr = torch.empty(1, dtype=torch.int32).pin_memory()
+
+    def e2e_step():
+        dc.copy_(hc, non_blocking=True)
+        dp.copy_(hp, non_blocking=True)
+        call(dc, dp)
+        hd.copy_(d, non_blocking=True)
+        hr.copy_(r, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = dist.max(a.elapsed_time(b) / 1e3, dev)
+
+    peaks, peaks_kind = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    traffic = profiled_traffic(w.name, kind="residual_diff")
+    clocks = sampler.summary(physical_gpu_index(dist.local_rank)) if dist.rank == 0 else {}
+    line = {
+        "metric": DIFF_METRIC, "value": value, "unit": "GB/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * max_seconds / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": diff_config(w, n),
+        "e2e": {"value": nbytes * e2e_steps * dist.world / e2e_s / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": 4 * n, "d2h_bytes_per_step": 8, "steps": e2e_steps,
+                "result_matches_device": bool(float(hd.item()) == float(d.item()) and int(hr.item()) == int(r.item())),
+                "diff": float(hd.item()), "reuse": int(hr.item())},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"HBM copy, {peaks_kind}", "traffic": traffic,
+                     "kernel": "residual_diff_kernel", "bytes_per_launch": nbytes},
+        "clocks": clocks,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        rate, sn, dt = diff_oracle_rate(cur.cpu(), prev.cpu(), args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": f"fp64 numpy oracle on the first {sn} elements: {dt:.2f} s"}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, dist: Dist):
     import torch
     import attention_dit_attn_b200 as dit
@@ -629,7 +796,7 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["attention", "lse_merge"], default="attention")
+    ap.add_argument("--op", choices=["attention", "lse_merge", "residual_diff"], default="attention")
     ap.add_argument("--parts", type=int, default=2, help="lse_merge: number of partial results (ring degree)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -642,11 +809,12 @@ def main(argv=None):
     if args.impl == "reference":
         # The oracle runs on rank 0's host cores only; other ranks exit at once.
         if int(os.environ.get("RANK", "0")) == 0:
-            (run_merge_reference if args.op == "lse_merge" else run_reference)(args, Dist.single())
+            {"lse_merge": run_merge_reference, "residual_diff": run_diff_reference}.get(
+                args.op, run_reference)(args, Dist.single())
         return
     dist = Dist(args.gpus)
     try:
-        (run_merge if args.op == "lse_merge" else run_ours)(args, dist)
+        {"lse_merge": run_merge, "residual_diff": run_diff}.get(args.op, run_ours)(args, dist)
     finally:
         dist.close()
 

@@ -27,6 +27,7 @@
 #ifndef DIT_ATTN_H
 #define DIT_ATTN_H
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -165,6 +166,52 @@ int dit_attn_launches_per_call(int B, int H, int L, int D, int dtype);
  */
 int dit_attn_lse_merge(const void *const *o_parts, const float *const *lse_parts, int n_parts,
                        void *o, float *lse, long long rows, int D, cudaStream_t stream);
+
+/*
+ * dit_attn_residual_diff_workspace_bytes — bytes of device workspace that
+ * dit_attn_residual_diff needs for n elements (0 if n < 1).  At most
+ * 16 + 16 * 1184 bytes.
+ */
+size_t dit_attn_residual_diff_workspace_bytes(long long n);
+
+/*
+ * dit_attn_residual_diff — the step-cache reuse decision, asynchronous on
+ * `stream`.
+ *
+ * Step caching (DBCache) reuses transformer work from the previous denoising
+ * step when the residual of the first blocks has changed little, against a
+ * `residual diff threshold` (0.12 in the published setting): page "How to
+ * Scale Diffusion Inference Across AMD RDNA 4 GPUs", section "Skip
+ * Transformer Work Only When the Model Has Enough Steps".  The page gives no
+ * formula; this computes the relative L1 change
+ *
+ *     diff = sum_i |cur_i - prev_i| / sum_i |prev_i|    (0/0 = 0, x/0 = +inf)
+ *     reuse = diff < threshold
+ *
+ * in one pass (fp32 per thread, fp64 across threads and blocks, summed in a
+ * fixed order, so repeated calls give identical results).
+ *
+ * cur, prev      device pointers to n bf16 values each (the residual of the
+ *                current and of the previous step), 16-byte aligned.
+ * n              1 <= n < 2^40.
+ * threshold      the reuse threshold; not NaN.
+ * workspace      device buffer of at least
+ *                dit_attn_residual_diff_workspace_bytes(n) bytes, 16-byte
+ *                aligned, zero-filled before its first use; each call leaves
+ *                it zeroed again.  Calls sharing a workspace must be ordered
+ *                (one stream).
+ * diff_out       device pointer to one fp32 (diff), or NULL.
+ * reuse_out      device pointer to one int32 (1 = reuse, 0 = compute), or NULL;
+ *                not both NULL.
+ *
+ * Ownership: the caller owns every buffer.  Errors (before anything is
+ * enqueued): DIT_ATTN_ERR_NULL, _SHAPE (n out of range or workspace too
+ * small), _ALIGN, _VALUE (NaN threshold), _ARCH; DIT_ATTN_ERR_LAUNCH if the
+ * launch fails.  The kernel has no waits.
+ */
+int dit_attn_residual_diff(const void *cur, const void *prev, long long n, float threshold,
+                           void *workspace, size_t workspace_bytes, float *diff_out, int *reuse_out,
+                           cudaStream_t stream);
 
 #ifdef __cplusplus
 }

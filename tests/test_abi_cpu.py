@@ -18,7 +18,8 @@ def test_library_exports_every_header_function(L):
     names = dit.header_functions()
     assert set(names) == {"dit_attn_fwd", "dit_attn_status_string", "dit_attn_check_device_error",
                           "dit_attn_set_wait_limit_ns", "dit_attn_selftest_wait_timeout",
-                          "dit_attn_launches_per_call", "dit_attn_lse_merge"}
+                          "dit_attn_launches_per_call", "dit_attn_lse_merge", "dit_attn_residual_diff",
+                          "dit_attn_residual_diff_workspace_bytes"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -94,3 +95,25 @@ def test_lse_merge_wellformed_call_without_gpu_reports_arch(L):
 
 def test_lse_merge_zero_rows_is_a_no_op_even_with_null_buffers(L):
     assert dit.dit_attn_lse_merge_ptr([0, 0], [0, 0], 0, None, 0, 128) == 0
+
+
+def test_residual_diff_workspace_size(L):
+    assert dit.dit_attn_residual_diff_workspace_bytes(0) == 0
+    assert dit.dit_attn_residual_diff_workspace_bytes(1) == 16 + 16
+    big = dit.dit_attn_residual_diff_workspace_bytes(1 << 34)
+    assert big == 16 + 16 * 1184
+
+
+@pytest.mark.parametrize("args,want", [
+    ((0, 16, 64, 0.12, 16, 64, 16, 16), 1),              # cur NULL
+    ((16, 16, 64, 0.12, 0, 64, 16, 16), 1),              # workspace NULL
+    ((16, 16, 64, 0.12, 16, 64, None, None), 1),         # no output at all
+    ((16, 16, 0, 0.12, 16, 64, 16, 16), 2),              # n < 1
+    ((16, 16, 64, 0.12, 16, 8, 16, 16), 2),              # workspace too small
+    ((24, 16, 64, 0.12, 16, 64, 16, 16), 4),             # cur not 16-byte aligned
+    ((16, 16, 64, 0.12, 16, 64, 18, 16), 4),             # diff_out not 4-byte aligned
+    ((16, 16, 64, float("nan"), 16, 64, 16, 16), 8),     # NaN threshold
+    ((16, 16, 64, 0.12, 16, 64, 16, 16), 5),             # well-formed: no GPU here
+])
+def test_residual_diff_argument_validation(L, args, want):
+    assert dit.dit_attn_residual_diff_ptr(*args) == want
