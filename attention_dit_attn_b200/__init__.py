@@ -25,7 +25,8 @@ __all__ = [
     "dit_attn_status_string", "dit_attn_check_device_error", "dit_attn_set_wait_limit_ns",
     "dit_attn_selftest_wait_timeout", "dit_attn_launches_per_call", "dit_attn_lse_merge",
     "dit_attn_lse_merge_ptr", "DIT_ATTN_MERGE_MAX_PARTS", "dit_attn_residual_diff",
-    "dit_attn_residual_diff_ptr", "dit_attn_residual_diff_workspace_bytes", "ensure_built", "lib",
+    "dit_attn_residual_diff_ptr", "dit_attn_residual_diff_workspace_bytes", "dit_attn_residual_diff_noalloc",
+    "ensure_built", "lib",
     "header_functions", "STATUS",
 ]
 
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.dit_attn_residual_diff.restype = i32
         L.dit_attn_residual_diff.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_float, vp, ctypes.c_size_t,
                                              vp, vp, vp]
+        L.dit_attn_residual_diff_noalloc.restype = i32
+        L.dit_attn_residual_diff_noalloc.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_float, vp, vp, vp]
         L.dit_attn_lse_merge.restype = i32
         L.dit_attn_lse_merge.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i32, vp, vp,
                                          ctypes.c_longlong, i32, vp]
@@ -271,4 +274,25 @@ def dit_attn_residual_diff(cur, prev, threshold: float = 0.12, *, workspace=None
                                     workspace.numel(), diff.data_ptr(), reuse.data_ptr(), _stream_handle(stream))
     if rc != 0:
         raise DitAttnError(rc, "dit_attn_residual_diff: ")
+    return diff, reuse
+
+
+def dit_attn_residual_diff_noalloc(cur, prev, threshold: float = 0.12, *, diff=None, reuse=None, stream=None):
+    """dit_attn_residual_diff without a workspace: the library's fixed device scratch is
+    used (calls on one device must be ordered).  Returns one-element fp32 / int32 CUDA
+    tensors (allocated here when not given; the C call itself allocates nothing)."""
+    import torch
+    for name, t in (("cur", cur), ("prev", prev)):
+        if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if cur.numel() != prev.numel():
+        raise ValueError("cur and prev must have the same number of elements")
+    if diff is None:
+        diff = torch.empty(1, dtype=torch.float32, device=cur.device)
+    if reuse is None:
+        reuse = torch.empty(1, dtype=torch.int32, device=cur.device)
+    rc = lib().dit_attn_residual_diff_noalloc(cur.data_ptr(), prev.data_ptr(), cur.numel(), ctypes.c_float(threshold),
+                                              diff.data_ptr(), reuse.data_ptr(), _stream_handle(stream))
+    if rc != 0:
+        raise DitAttnError(rc, "dit_attn_residual_diff_noalloc: ")
     return diff, reuse

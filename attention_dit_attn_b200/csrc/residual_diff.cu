@@ -155,6 +155,15 @@ int blocks_for(long long n, int resident)
 
 std::atomic<int> g_resident{0};
 
+// Scratch of the no-allocation entry point: the largest workspace any n needs,
+// in the module's own device memory (zero at load; every call leaves it zero).
+constexpr size_t kScratchBytes = kHeaderBytes + sizeof(double2) * kMaxBlocks;
+static __device__ __align__(256) unsigned char g_diff_scratch[kScratchBytes];
+
+// Its address per device, looked up once.
+constexpr int kMaxDevices = 64;
+std::atomic<void *> g_scratch_addr[kMaxDevices];
+
 bool aligned(const void *q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) == 0; }
 
 } // namespace
@@ -208,4 +217,21 @@ extern "C" int dit_attn_residual_diff(const void *cur, const void *prev, long lo
     p.reuse_out = reuse_out;
     residual_diff_kernel<<<blocks_for(n, resident), kThreads, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? DIT_ATTN_OK : DIT_ATTN_ERR_LAUNCH;
+}
+
+extern "C" int dit_attn_residual_diff_noalloc(const void *cur, const void *prev, long long n, float threshold,
+                                              float *diff_out, int *reuse_out, cudaStream_t stream)
+{
+    if (n < 1 || n >= (1ll << 40) || dit_attn_residual_diff_workspace_bytes(n) > kScratchBytes)
+        return DIT_ATTN_ERR_SHAPE;
+    int device = 0;
+    if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices)
+        return DIT_ATTN_ERR_ARCH;
+    void *scratch = g_scratch_addr[device].load(std::memory_order_acquire);
+    if (scratch == nullptr) {
+        if (cudaGetSymbolAddress(&scratch, g_diff_scratch) != cudaSuccess)
+            return DIT_ATTN_ERR_ARCH;
+        g_scratch_addr[device].store(scratch, std::memory_order_release);
+    }
+    return dit_attn_residual_diff(cur, prev, n, threshold, scratch, kScratchBytes, diff_out, reuse_out, stream);
 }

@@ -213,6 +213,24 @@ int dit_attn_residual_diff(const void *cur, const void *prev, long long n, float
                            void *workspace, size_t workspace_bytes, float *diff_out, int *reuse_out,
                            cudaStream_t stream);
 
+/*
+ * dit_attn_residual_diff_noalloc — dit_attn_residual_diff without a caller
+ * workspace and without allocating anything: the scratch is a fixed array in
+ * the library's own device memory (zero at load, left zero by every call),
+ * whose address is looked up once per device.  The pages have no counterpart
+ * of this entry point; it exists so that a caller with no allocator at hand
+ * (e.g. a captured CUDA graph built before any buffer is known) can take the
+ * step-cache decision.
+ *
+ * Same arguments, results and errors as dit_attn_residual_diff, minus the
+ * workspace.  n above what the fixed scratch covers is rejected with
+ * DIT_ATTN_ERR_SHAPE (the scratch covers every n < 2^40).  Because the scratch
+ * is shared, calls on one device must be ordered (one stream, or streams
+ * ordered by events); concurrent calls would race on it.
+ */
+int dit_attn_residual_diff_noalloc(const void *cur, const void *prev, long long n, float threshold,
+                                   float *diff_out, int *reuse_out, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,7 @@ def test_library_exports_every_header_function(L):
     assert set(names) == {"dit_attn_fwd", "dit_attn_status_string", "dit_attn_check_device_error",
                           "dit_attn_set_wait_limit_ns", "dit_attn_selftest_wait_timeout",
                           "dit_attn_launches_per_call", "dit_attn_lse_merge", "dit_attn_residual_diff",
-                          "dit_attn_residual_diff_workspace_bytes"}
+                          "dit_attn_residual_diff_workspace_bytes", "dit_attn_residual_diff_noalloc"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -117,3 +117,13 @@ def test_residual_diff_workspace_size(L):
 ])
 def test_residual_diff_argument_validation(L, args, want):
     assert dit.dit_attn_residual_diff_ptr(*args) == want
+
+
+def test_residual_diff_noalloc_rejects_sizes_before_any_cuda_call(L):
+    L.dit_attn_residual_diff_noalloc.restype = ctypes.c_int
+    L.dit_attn_residual_diff_noalloc.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong,
+                                                 ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    assert L.dit_attn_residual_diff_noalloc(16, 16, 0, ctypes.c_float(0.12), 16, 16, None) == 2
+    assert L.dit_attn_residual_diff_noalloc(16, 16, 1 << 40, ctypes.c_float(0.12), 16, 16, None) == 2
+    # well-formed: reaches the device query, which fails here without a GPU
+    assert L.dit_attn_residual_diff_noalloc(16, 16, 64, ctypes.c_float(0.12), 16, 16, None) == 5
