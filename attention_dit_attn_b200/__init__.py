@@ -26,6 +26,7 @@ __all__ = [
     "dit_attn_selftest_wait_timeout", "dit_attn_launches_per_call", "dit_attn_lse_merge",
     "dit_attn_lse_merge_ptr", "DIT_ATTN_MERGE_MAX_PARTS", "dit_attn_residual_diff",
     "dit_attn_residual_diff_ptr", "dit_attn_residual_diff_workspace_bytes", "dit_attn_residual_diff_noalloc",
+    "dit_attn_mxfp4_quantize", "dit_attn_mxfp4_quantize_ptr",
     "ensure_built", "lib",
     "header_functions", "STATUS",
 ]
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
                                              vp, vp, vp]
         L.dit_attn_residual_diff_noalloc.restype = i32
         L.dit_attn_residual_diff_noalloc.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_float, vp, vp, vp]
+        L.dit_attn_mxfp4_quantize.restype = i32
+        L.dit_attn_mxfp4_quantize.argtypes = [vp, vp, vp, ctypes.c_longlong, i32, vp]
         L.dit_attn_lse_merge.restype = i32
         L.dit_attn_lse_merge.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i32, vp, vp,
                                          ctypes.c_longlong, i32, vp]
@@ -296,3 +299,30 @@ def dit_attn_residual_diff_noalloc(cur, prev, threshold: float = 0.12, *, diff=N
     if rc != 0:
         raise DitAttnError(rc, "dit_attn_residual_diff_noalloc: ")
     return diff, reuse
+
+
+def dit_attn_mxfp4_quantize_ptr(x: int, q: int, scales: int, rows: int, K: int, stream: int = 0) -> int:
+    """Raw C-ABI call with integer device pointers; returns the status code."""
+    return lib().dit_attn_mxfp4_quantize(x, q, scales, rows, K, stream)
+
+
+def dit_attn_mxfp4_quantize(x, q=None, scales=None, *, stream=None):
+    """MXFP4 (1x32 blocks) quantisation of a bf16 CUDA tensor [..., K] (K % 32 == 0).
+    Returns (q uint8 [..., K/2] packed E2M1 codes, scales uint8 [..., K/32] E8M0)."""
+    import torch
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous()):
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    K = x.shape[-1]
+    rows = x.numel() // K if K else 0
+    lead = tuple(x.shape[:-1])
+    if q is None:
+        q = torch.empty(lead + (K // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(lead + (K // 32,), dtype=torch.uint8, device=x.device)
+    for name, t, cols in (("q", q, K // 2), ("scales", scales, K // 32)):
+        if not (t.is_cuda and t.dtype == torch.uint8 and t.is_contiguous() and t.numel() == rows * cols):
+            raise ValueError(f"{name} must be a contiguous uint8 CUDA tensor with {rows * cols} elements")
+    rc = dit_attn_mxfp4_quantize_ptr(x.data_ptr(), q.data_ptr(), scales.data_ptr(), rows, K, _stream_handle(stream))
+    if rc != 0:
+        raise DitAttnError(rc, "dit_attn_mxfp4_quantize: ")
+    return q, scales

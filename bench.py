@@ -24,6 +24,8 @@ hot path is one kernel launch).  Prints ONE JSON line on rank 0.
 * --op residual_diff: the step-cache reuse decision (relative L1 change of a
   hidden-state-sized bf16 residual, B*L*H*D elements of the workload, against
   the previous step's); GB/s of algorithmic HBM traffic.
+* --op mxfp4_quant: the MXFP4 1x32 activation quantiser on a (B*L) x (H*D)
+  bf16 activation of the workload; GB/s of algorithmic HBM traffic.
 Multi-GPU (torchrun): every rank runs its own replica (no data exchange:
 heads and batches are independent), scaling "weak".
 """
@@ -46,6 +48,7 @@ sys.path.insert(0, ROOT)
 METRIC = "attention TFLOP/s and % of B200 tensor-core peak at 1 GPU"
 MERGE_METRIC = "LSE merge of partial attentions: GB/s of algorithmic HBM traffic at 1 GPU"
 DIFF_METRIC = "step-cache residual-change decision: GB/s of algorithmic HBM traffic at 1 GPU"
+MXFP4_METRIC = "MXFP4 1x32 activation quantiser: GB/s of algorithmic HBM traffic at 1 GPU"
 DEFAULT_WORKLOAD = "flux_2048_cfg"      # the first workload with L >= 16k (the stated target)
 NOMINAL_TFLOPS = {"bf16": 2250.0, "e4m3": 4500.0}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
@@ -69,6 +72,7 @@ KERNEL_SOURCES = {
     "attn_fwd": ["attn_common.cuh", "attn_fwd_sm100.cuh", "dit_attn.cu", "exp2_poly_fit.py", "sm100_ptx.cuh"],
     "lse_merge": ["lse_merge.cu"],
     "residual_diff": ["residual_diff.cu"],
+    "mxfp4_quant": ["mxfp4_quant.cu"],
 }
 
 
@@ -647,6 +651,157 @@ def run_diff(args, dist: Dist):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ MXFP4 activation quantiser
+
+def mxfp4_bytes(rows: int, K: int) -> int:
+    return rows * (2 * K + K // 2 + K // 32)
+
+
+def mxfp4_config(w, rows, K):
+    return {"workload": w.name, "op": "mxfp4_quant", "rows": rows, "K": K, "input_dtype": "bf16",
+            "output": "E2M1 codes (K/2 bytes per row) + E8M0 scales (K/32 bytes per row)",
+            "bytes_per_call": mxfp4_bytes(rows, K),
+            "l2": "inputs larger than L2" if 2 * rows * K > L2_BYTES else "L2 flushed between timed steps (256 MB write)",
+            "parallelism": "replicas"}
+
+
+def mxfp4_oracle_rate(x_cpu, seconds: float):
+    from oracle import mxfp4
+    rows = 8
+    K = x_cpu.shape[1]
+    while True:
+        xs = x_cpu[:rows].double().numpy()
+        t0 = time.perf_counter()
+        mxfp4.quantize(xs)
+        dt = time.perf_counter() - t0
+        if dt >= seconds / 4 or rows >= x_cpu.shape[0]:
+            return mxfp4_bytes(rows, K) / dt / 1e9, rows, dt
+        rows = min(x_cpu.shape[0], rows * 4)
+
+
+def run_mxfp4_reference(args, dist: Dist):
+    if dist.rank != 0:
+        return
+    import torch
+    from attention_dit_attn_b200 import workloads as wl
+    w = wl.ALL[args.workload]
+    rows, K = w.B * w.L, w.H * w.D
+    g = torch.Generator().manual_seed(w.seed)
+    x = torch.randn((min(rows, 4096), K), generator=g).to(torch.bfloat16)
+    per = 60.0 / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        mxfp4_oracle_rate(x, per)
+    rates = [mxfp4_oracle_rate(x, per) for _ in range(args.steps)]
+    value = statistics.median(r[0] for r in rates)
+    line = {
+        "impl": "reference", "metric": MXFP4_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * mxfp4_bytes(rows, K) / (value * 1e9),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": mxfp4_config(w, rows, K),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: fp64 numpy oracle on {rates[0][1]} rows of {K}"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_mxfp4(args, dist: Dist):
+    import torch
+    import attention_dit_attn_b200 as dit
+    from attention_dit_attn_b200 import workloads as wl
+
+    dit.ensure_built()
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    w = wl.ALL[args.workload]
+    rows, K = w.B * w.L, w.H * w.D
+    g = torch.Generator(device=dev).manual_seed(w.seed)
+    x = torch.randn((rows, K), generator=g, device=dev).to(torch.bfloat16)
+    q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev)
+    sc = torch.empty((rows, K // 32), dtype=torch.uint8, device=dev)
+    nbytes = mxfp4_bytes(rows, K)
+    flush = None
+    if 2 * rows * K <= L2_BYTES:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda xx: dit.dit_attn_mxfp4_quantize(xx, q, sc, stream=stream)
+    for _ in range(args.warmup):
+        call(x)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler()
+    if dist.rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in evs:
+        if flush is not None:
+            flush.fill_(1)
+        a.record(stream)
+        call(x)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    seconds = sum(a.elapsed_time(b) for a, b in evs) / 1e3
+    dist.barrier()
+    if dist.rank == 0:
+        time.sleep(0.2)
+        sampler.stop()
+    max_seconds = dist.max(seconds, dev)
+    value = nbytes * args.steps * dist.world / max_seconds / 1e9
+    achieved = nbytes / (seconds / args.steps) / 1e9
+
+    e2e_steps = max(3, min(args.steps, 10))
+    hx = x.cpu().pin_memory()
+    dx = torch.empty_like(x)
+    hq = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    hs = torch.empty(sc.shape, dtype=sc.dtype).pin_memory()
+
+    def e2e_step():
+        dx.copy_(hx, non_blocking=True)
+        call(dx)
+        hq.copy_(q, non_blocking=True)
+        hs.copy_(sc, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = dist.max(a.elapsed_time(b) / 1e3, dev)
+
+    peaks, peaks_kind = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    traffic = profiled_traffic(w.name, kind="mxfp4_quant")
+    clocks = sampler.summary(physical_gpu_index(dist.local_rank)) if dist.rank == 0 else {}
+    line = {
+        "metric": MXFP4_METRIC, "value": value, "unit": "GB/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * max_seconds / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": mxfp4_config(w, rows, K),
+        "e2e": {"value": nbytes * e2e_steps * dist.world / e2e_s / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": 2 * rows * K, "d2h_bytes_per_step": rows * (K // 2 + K // 32),
+                "steps": e2e_steps, "result_matches_device": bool(torch.equal(hq, q.cpu()) and torch.equal(hs, sc.cpu()))},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"HBM copy, {peaks_kind}", "traffic": traffic,
+                     "kernel": "mxfp4_quant_kernel", "bytes_per_launch": nbytes},
+        "clocks": clocks,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        rate, srows, dt = mxfp4_oracle_rate(x[:4096].cpu(), args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": f"fp64 numpy oracle on the first {srows} rows of {K}: {dt:.2f} s"}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, dist: Dist):
     import torch
     import attention_dit_attn_b200 as dit
@@ -796,7 +951,7 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["attention", "lse_merge", "residual_diff"], default="attention")
+    ap.add_argument("--op", choices=["attention", "lse_merge", "residual_diff", "mxfp4_quant"], default="attention")
     ap.add_argument("--parts", type=int, default=2, help="lse_merge: number of partial results (ring degree)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -809,12 +964,14 @@ def main(argv=None):
     if args.impl == "reference":
         # The oracle runs on rank 0's host cores only; other ranks exit at once.
         if int(os.environ.get("RANK", "0")) == 0:
-            {"lse_merge": run_merge_reference, "residual_diff": run_diff_reference}.get(
+            {"lse_merge": run_merge_reference, "residual_diff": run_diff_reference,
+             "mxfp4_quant": run_mxfp4_reference}.get(
                 args.op, run_reference)(args, Dist.single())
         return
     dist = Dist(args.gpus)
     try:
-        {"lse_merge": run_merge, "residual_diff": run_diff}.get(args.op, run_ours)(args, dist)
+        {"lse_merge": run_merge, "residual_diff": run_diff, "mxfp4_quant": run_mxfp4}.get(
+            args.op, run_ours)(args, dist)
     finally:
         dist.close()
 

@@ -214,6 +214,32 @@ int dit_attn_residual_diff(const void *cur, const void *prev, long long n, float
                            cudaStream_t stream);
 
 /*
+ * dit_attn_mxfp4_quantize — MXFP4 (OCP Microscaling, 1x32 blocks) quantiser
+ * of bf16 activations, asynchronous on `stream`.
+ *
+ * The page "Accelerating Diffusers and xDiT Image Generation with MXFP4 using
+ * AMD Quark on AMD Instinct MI350 GPUs" (sections "MXFP4 Quantization",
+ * "MXFP4 Kernel") quantises linear-layer activations on the fly to MXFP4:
+ * 32 consecutive values along a row share one E8M0 scale and each is a 4-bit
+ * E2M1 float.  The page does not restate the rule; the OCP MX definition it
+ * cites is used: per block, s = clamp(floor(log2 max|v|) - 2, -127, 127)
+ * (-127 for a zero block), q_i = E2M1(v_i / 2^s) rounded to nearest even and
+ * saturated at +-6, with the sign kept (-0 included).
+ *
+ * x       device pointer, bf16 [rows, K] row-major, 16-byte aligned.  Finite
+ *         values only (non-finite inputs give unspecified codes).
+ * q       device pointer, uint8 [rows, K/2]: two codes per byte, the first
+ *         element of each pair in bits 0..3; 16-byte aligned.
+ * scales  device pointer, uint8 [rows, K/32]: the E8M0 byte s + 127 per block.
+ * rows    >= 0 (0: nothing is enqueued, pointers unused); rows * K < 2^40.
+ * K       a multiple of 32.
+ *
+ * Errors (before anything is enqueued): DIT_ATTN_ERR_SHAPE, _NULL, _ALIGN,
+ * _ARCH; DIT_ATTN_ERR_LAUNCH if the launch fails.  The kernel has no waits.
+ */
+int dit_attn_mxfp4_quantize(const void *x, void *q, void *scales, long long rows, int K, cudaStream_t stream);
+
+/*
  * dit_attn_residual_diff_noalloc — dit_attn_residual_diff without a caller
  * workspace and without allocating anything: the scratch is a fixed array in
  * the library's own device memory (zero at load, left zero by every call),

@@ -19,7 +19,8 @@ def test_library_exports_every_header_function(L):
     assert set(names) == {"dit_attn_fwd", "dit_attn_status_string", "dit_attn_check_device_error",
                           "dit_attn_set_wait_limit_ns", "dit_attn_selftest_wait_timeout",
                           "dit_attn_launches_per_call", "dit_attn_lse_merge", "dit_attn_residual_diff",
-                          "dit_attn_residual_diff_workspace_bytes", "dit_attn_residual_diff_noalloc"}
+                          "dit_attn_residual_diff_workspace_bytes", "dit_attn_residual_diff_noalloc",
+                          "dit_attn_mxfp4_quantize"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -127,3 +128,16 @@ def test_residual_diff_noalloc_rejects_sizes_before_any_cuda_call(L):
     assert L.dit_attn_residual_diff_noalloc(16, 16, 1 << 40, ctypes.c_float(0.12), 16, 16, None) == 2
     # well-formed: reaches the device query, which fails here without a GPU
     assert L.dit_attn_residual_diff_noalloc(16, 16, 64, ctypes.c_float(0.12), 16, 16, None) == 5
+
+
+@pytest.mark.parametrize("args,want", [
+    ((16, 16, 16, 4, 48), 2),            # K not a multiple of 32
+    ((16, 16, 16, 4, 0), 2),             # K = 0
+    ((16, 16, 16, -1, 64), 2),           # negative rows
+    ((0, 0, 0, 0, 64), 0),               # zero rows: no-op, pointers unused
+    ((0, 16, 16, 4, 64), 1),             # x NULL
+    ((24, 16, 16, 4, 64), 4),            # x not 16-byte aligned
+    ((16, 16, 16, 4, 64), 5),            # well-formed: no GPU here
+])
+def test_mxfp4_quantize_argument_validation(L, args, want):
+    assert dit.dit_attn_mxfp4_quantize_ptr(*args) == want
