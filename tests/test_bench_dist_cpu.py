@@ -76,3 +76,16 @@ def test_bench_rejects_too_few_warmup_steps():
     r = subprocess.run([sys.executable, "bench.py", "--warmup", "2"], cwd=ROOT, capture_output=True,
                        text=True, timeout=120)
     assert r.returncode != 0
+
+
+@pytest.mark.parametrize("op,unit", [("lse_merge", "GB/s"), ("residual_diff", "GB/s"), ("mxfp4_quant", "GB/s")])
+def test_reference_arm_of_each_op_prints_one_json_line(op, unit):
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--op", op, "--workload", "tiny_256",
+                        "--steps", "3", "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == unit and d["value"] > 0
+    assert d["config"]["op"] == op and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
