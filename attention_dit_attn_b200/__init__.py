@@ -26,7 +26,8 @@ __all__ = [
     "dit_attn_selftest_wait_timeout", "dit_attn_launches_per_call", "dit_attn_lse_merge",
     "dit_attn_lse_merge_ptr", "DIT_ATTN_MERGE_MAX_PARTS", "dit_attn_residual_diff",
     "dit_attn_residual_diff_ptr", "dit_attn_residual_diff_workspace_bytes", "dit_attn_residual_diff_noalloc",
-    "dit_attn_mxfp4_quantize", "dit_attn_mxfp4_quantize_ptr",
+    "dit_attn_mxfp4_quantize", "dit_attn_mxfp4_quantize_ptr", "dit_attn_block_transpose",
+    "dit_attn_absmax_rows", "dit_attn_quantize_e4m3_rows",
     "ensure_built", "lib",
     "header_functions", "STATUS",
 ]
@@ -87,6 +88,12 @@ def lib() -> ctypes.CDLL:
         L.dit_attn_residual_diff_noalloc.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_float, vp, vp, vp]
         L.dit_attn_mxfp4_quantize.restype = i32
         L.dit_attn_mxfp4_quantize.argtypes = [vp, vp, vp, ctypes.c_longlong, i32, vp]
+        L.dit_attn_block_transpose.restype = i32
+        L.dit_attn_block_transpose.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_longlong, ctypes.c_longlong, vp]
+        L.dit_attn_absmax_rows.restype = i32
+        L.dit_attn_absmax_rows.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_longlong, vp]
+        L.dit_attn_quantize_e4m3_rows.restype = i32
+        L.dit_attn_quantize_e4m3_rows.argtypes = [vp, vp, vp, vp, ctypes.c_longlong, ctypes.c_longlong, vp]
         L.dit_attn_lse_merge.restype = i32
         L.dit_attn_lse_merge.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i32, vp, vp,
                                          ctypes.c_longlong, i32, vp]
@@ -326,3 +333,53 @@ def dit_attn_mxfp4_quantize(x, q=None, scales=None, *, stream=None):
     if rc != 0:
         raise DitAttnError(rc, "dit_attn_mxfp4_quantize: ")
     return q, scales
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise DitAttnError(rc, what + ": ")
+
+
+def dit_attn_block_transpose(x, R: int, C: int, out=None, *, stream=None):
+    """out[c][r] = x[r][c] over an R x C grid of equal contiguous blocks of a CUDA tensor
+    (its bytes split into R*C blocks).  Returns a tensor of x's dtype and numel."""
+    import torch
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.is_contiguous()):
+        raise ValueError("x must be a contiguous CUDA tensor")
+    nbytes = x.numel() * x.element_size()
+    if R * C == 0 or nbytes % (R * C):
+        raise ValueError("x's bytes must split into R*C equal blocks")
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().dit_attn_block_transpose(x.data_ptr(), out.data_ptr(), R, C, nbytes // (R * C),
+                                          _stream_handle(stream)), "dit_attn_block_transpose")
+    return out
+
+
+def dit_attn_absmax_rows(x, rows: int, out=None, *, stream=None):
+    """max |x| of each of `rows` equal rows of a bf16 CUDA tensor -> fp32 [rows]."""
+    import torch
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous()):
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    if out is None:
+        out = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(lib().dit_attn_absmax_rows(x.data_ptr(), out.data_ptr(), rows, x.numel() // max(rows, 1),
+                                      _stream_handle(stream)), "dit_attn_absmax_rows")
+    return out
+
+
+def dit_attn_quantize_e4m3_rows(x, amax, q=None, scale=None, *, stream=None):
+    """e4m3(x / (amax / 448)) per row (rows = amax.numel()); returns (q float8_e4m3fn like x,
+    fp32 dequantisation scales [rows])."""
+    import torch
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous()):
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    rows = amax.numel()
+    if q is None:
+        q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    if scale is None:
+        scale = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(lib().dit_attn_quantize_e4m3_rows(x.data_ptr(), amax.data_ptr(), q.data_ptr(), scale.data_ptr(), rows,
+                                             x.numel() // max(rows, 1), _stream_handle(stream)),
+           "dit_attn_quantize_e4m3_rows")
+    return q, scale

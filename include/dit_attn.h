@@ -240,6 +240,43 @@ int dit_attn_residual_diff(const void *cur, const void *prev, long long n, float
 int dit_attn_mxfp4_quantize(const void *x, void *q, void *scales, long long rows, int K, cudaStream_t stream);
 
 /*
+ * Local data movement of Ulysses sequence parallelism (page "How to Scale
+ * Diffusion Inference Across AMD RDNA 4 GPUs", section "Balance Transformer
+ * Work and Communication": tokens are divided across GPUs and every attention
+ * layer exchanges data with an all-to-all; `--use fp8 comms` sends it in
+ * FP8).  The exchange itself is a collective of the caller's (NCCL); these
+ * three calls are the per-GPU steps around it.  All asynchronous on
+ * `stream`; argument errors are returned before anything is enqueued; no
+ * waits on the device.
+ *
+ * dit_attn_block_transpose — out[c][r] = in[r][c] for an R x C grid of
+ * contiguous blocks of block_bytes each (a multiple of 4; 16 with 16-byte
+ * aligned pointers takes 16-byte copies).  in and out must not overlap.
+ * R, C, block_bytes >= 0 (any 0: nothing is enqueued, pointers unused);
+ * R * C * block_bytes <= 2^40.
+ */
+int dit_attn_block_transpose(const void *in, void *out, long long R, long long C, long long block_bytes,
+                             cudaStream_t stream);
+
+/*
+ * dit_attn_absmax_rows — amax[r] = max_i |x[r][i]| (fp32) for bf16 rows of
+ * row_len values (a multiple of 8), e.g. rows = B*H of a [B, H, Ls, D] shard.
+ * x 16-byte aligned.  rows = 0: nothing is enqueued.
+ */
+int dit_attn_absmax_rows(const void *x, float *amax, long long rows, long long row_len, cudaStream_t stream);
+
+/*
+ * dit_attn_quantize_e4m3_rows — per row r, with s = amax[r] / 448 (fp32,
+ * correctly rounded; 1 if amax[r] == 0): q[r][i] = E4M3(x[r][i] / s), the
+ * quotient correctly rounded in fp32, then rounded to nearest even and
+ * saturated at +-448 (OCP FP8 E4M3).  scale_out[r] = s (the dequantisation
+ * scale dit_attn_fwd takes), or NULL.  row_len a multiple of 16; x and q
+ * 16-byte aligned.  rows = 0: nothing is enqueued.
+ */
+int dit_attn_quantize_e4m3_rows(const void *x, const float *amax, void *q, float *scale_out, long long rows,
+                                long long row_len, cudaStream_t stream);
+
+/*
  * dit_attn_residual_diff_noalloc — dit_attn_residual_diff without a caller
  * workspace and without allocating anything: the scratch is a fixed array in
  * the library's own device memory (zero at load, left zero by every call),

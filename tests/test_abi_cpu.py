@@ -20,7 +20,8 @@ def test_library_exports_every_header_function(L):
                           "dit_attn_set_wait_limit_ns", "dit_attn_selftest_wait_timeout",
                           "dit_attn_launches_per_call", "dit_attn_lse_merge", "dit_attn_residual_diff",
                           "dit_attn_residual_diff_workspace_bytes", "dit_attn_residual_diff_noalloc",
-                          "dit_attn_mxfp4_quantize"}
+                          "dit_attn_mxfp4_quantize", "dit_attn_block_transpose", "dit_attn_absmax_rows",
+                          "dit_attn_quantize_e4m3_rows"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -141,3 +142,23 @@ def test_residual_diff_noalloc_rejects_sizes_before_any_cuda_call(L):
 ])
 def test_mxfp4_quantize_argument_validation(L, args, want):
     assert dit.dit_attn_mxfp4_quantize_ptr(*args) == want
+
+
+def test_ulysses_ops_argument_validation(L):
+    vp = ctypes.c_void_p
+    L.dit_attn_block_transpose.restype = ctypes.c_int
+    L.dit_attn_block_transpose.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_longlong, ctypes.c_longlong, vp]
+    L.dit_attn_absmax_rows.restype = ctypes.c_int
+    L.dit_attn_absmax_rows.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_longlong, vp]
+    L.dit_attn_quantize_e4m3_rows.restype = ctypes.c_int
+    L.dit_attn_quantize_e4m3_rows.argtypes = [vp, vp, vp, vp, ctypes.c_longlong, ctypes.c_longlong, vp]
+    assert L.dit_attn_block_transpose(16, 32, 2, 3, 6, None) == 2          # block bytes not a multiple of 4
+    assert L.dit_attn_block_transpose(None, None, 0, 3, 16, None) == 0      # empty: no-op
+    assert L.dit_attn_block_transpose(None, 32, 2, 3, 16, None) == 1
+    assert L.dit_attn_block_transpose(18, 32, 2, 3, 16, None) == 4          # in not 4-byte aligned
+    assert L.dit_attn_block_transpose(16, 32, 2, 3, 16, None) == 5          # well-formed: no GPU here
+    assert L.dit_attn_absmax_rows(16, 16, 4, 12, None) == 2                 # row_len not a multiple of 8
+    assert L.dit_attn_absmax_rows(16, 16, 4, 64, None) == 5
+    assert L.dit_attn_quantize_e4m3_rows(16, 16, 16, None, 4, 24, None) == 2   # row_len not a multiple of 16
+    assert L.dit_attn_quantize_e4m3_rows(16, 16, None, None, 4, 64, None) == 1
+    assert L.dit_attn_quantize_e4m3_rows(16, 16, 16, None, 4, 64, None) == 5
