@@ -27,6 +27,8 @@ SMALL = [
     (1, 1, 2, 64, "bf16"),
     (1, 2, 700, 64, "bf16"),
     (3, 2, 385, 64, "bf16"),
+    (1, 1, 33, 64, "bf16"),             # D = 64: four key splits, one key in the second
+    (1, 2, 353, 64, "e4m3"),            # last tile: splits 0-2 valid, split 3 one key
     (1, 1, 1, 64, "e4m3"),
     (2, 2, 300, 64, "e4m3"),
     (1, 2, 1000, 64, "e4m3"),
