@@ -15,7 +15,11 @@
 //    every rank quantises its shard with the same per-head scale, so the
 //    received FP8 tensors are exactly the inputs of the FP8 attention path.
 //
-// All three are memory-bound: 16-byte loads and stores, no waits.
+// All three are memory-bound: 16-byte loads and stores, no waits.  A row is
+// one head of a shard, so there are few rows (B H) of up to millions of
+// values: every kernel splits each row over many CTAs (grid.x = chunks of a
+// row, grid.y = rows), and the absmax CTAs combine their partial maxima with
+// an atomic max on the (order-preserving) bit patterns of non-negative floats.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -26,6 +30,8 @@
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kUnroll = 4;                               // units in flight per thread
+constexpr long long kUnitsPerCta = (long long)kUnroll * kThreads;
 constexpr float kE4M3Max = 448.f;
 
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
@@ -52,34 +58,44 @@ __global__ void __launch_bounds__(kThreads) block_transpose_kernel(const W *in, 
     }
 }
 
-// Per row: max |x| over row_len bf16 (row_len % 8 == 0), one CTA per row (grid-strided).
-__global__ void __launch_bounds__(kThreads) absmax_rows_kernel(const uint4 *x, float *amax, long long rows,
-                                                               long long vec_per_row)
+// Per row: max |x| over row_len bf16 (row_len % 8 == 0).  CTA (x, y) covers
+// vectors [x U, x U + U) (U = kUnitsPerCta, kUnroll per thread, all loads
+// issued before use) of rows y, y + gridDim.y, ...; amax_bits holds 0 on
+// entry and receives max(|bf16| bits) << 16, the float bits of the maximum.
+__global__ void __launch_bounds__(kThreads) absmax_rows_kernel(const uint4 *x, unsigned int *amax_bits,
+                                                               long long rows, long long vec_per_row)
 {
-    __shared__ float red[kThreads / 32];
-    for (long long row = blockIdx.x; row < rows; row += gridDim.x) {
+    __shared__ uint32_t red[kThreads / 32];
+    const long long beg = (long long)blockIdx.x * kUnitsPerCta + threadIdx.x;
+    for (long long row = blockIdx.y; row < rows; row += gridDim.y) {
         const uint4 *src = x + row * vec_per_row;
-        uint32_t m = 0;                                  // max of |bf16| bit patterns (order-preserving)
-        for (long long i = threadIdx.x; i < vec_per_row; i += kThreads) {
-            const uint4 w = ld_stream(src + i);
-            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+        uint4 w[kUnroll];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                m = max(m, u[k] & 0x7FFFu);
-                m = max(m, (u[k] >> 16) & 0x7FFFu);
+        for (int k = 0; k < kUnroll; ++k) {
+            const long long i = beg + (long long)k * kThreads;
+            w[k] = i < vec_per_row ? ld_stream(src + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        uint32_t m = 0;                                  // max of |bf16| bit patterns (order-preserving)
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            const uint32_t u[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                m = max(m, u[e] & 0x7FFFu);
+                m = max(m, (u[e] >> 16) & 0x7FFFu);
             }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
         if ((threadIdx.x & 31) == 0)
-            red[threadIdx.x >> 5] = __uint_as_float(m << 16);
+            red[threadIdx.x >> 5] = m;
         __syncthreads();
         if (threadIdx.x == 0) {
-            float r = 0.f;
+            uint32_t r = 0;
             for (int w = 0; w < kThreads / 32; ++w)
-                r = fmaxf(r, red[w]);
-            amax[row] = r;
+                r = max(r, red[w]);
+            atomicMax(amax_bits + row, r << 16);
         }
         __syncthreads();
     }
@@ -93,29 +109,45 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
 }
 
 // Per row: q = e4m3(x / s), s = amax / 448 (1 if amax == 0); 16 values per
-// thread-iteration (two 16-byte loads, one 16-byte store).
+// unit (two 16-byte loads, one 16-byte store).  CTA (x, y) covers units
+// [x U, x U + U) (kUnroll per thread, all loads issued before use) of rows
+// y, y + gridDim.y, ...; the CTAs with x = 0 write the row's scale.
 __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const uint4 *x, uint4 *q, const float *amax,
                                                                  float *scale_out, long long rows,
                                                                  long long vec16_per_row)
 {
-    for (long long row = blockIdx.x; row < rows; row += gridDim.x) {
+    const long long beg = (long long)blockIdx.x * kUnitsPerCta + threadIdx.x;
+    for (long long row = blockIdx.y; row < rows; row += gridDim.y) {
         const float a = amax[row];
         const float s = a > 0.f ? __fdiv_rn(a, kE4M3Max) : 1.f;
-        if (threadIdx.x == 0 && scale_out != nullptr)
+        if (blockIdx.x == 0 && threadIdx.x == 0 && scale_out != nullptr)
             scale_out[row] = s;
         const uint4 *src = x + row * vec16_per_row * 2;
         uint4 *dst = q + row * vec16_per_row;
-        for (long long i = threadIdx.x; i < vec16_per_row; i += kThreads) {
-            const uint4 w0 = ld_stream(src + 2 * i), w1 = ld_stream(src + 2 * i + 1);
+        uint4 w[2 * kUnroll];
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            const long long i = beg + (long long)k * kThreads;
+            if (i < vec16_per_row) {
+                w[2 * k] = ld_stream(src + 2 * i);
+                w[2 * k + 1] = ld_stream(src + 2 * i + 1);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            const long long i = beg + (long long)k * kThreads;
+            if (i >= vec16_per_row)
+                break;
+            const uint4 w0 = w[2 * k], w1 = w[2 * k + 1];
             const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
             uint32_t out[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float v0 = __fdiv_rn(__uint_as_float(u[2 * k] << 16), s);
-                const float v1 = __fdiv_rn(__uint_as_float(u[2 * k] & 0xFFFF0000u), s);
-                const float v2 = __fdiv_rn(__uint_as_float(u[2 * k + 1] << 16), s);
-                const float v3 = __fdiv_rn(__uint_as_float(u[2 * k + 1] & 0xFFFF0000u), s);
-                out[k] = e4m3x2(v0, v1) | (e4m3x2(v2, v3) << 16);
+            for (int e = 0; e < 4; ++e) {
+                const float v0 = __fdiv_rn(__uint_as_float(u[2 * e] << 16), s);
+                const float v1 = __fdiv_rn(__uint_as_float(u[2 * e] & 0xFFFF0000u), s);
+                const float v2 = __fdiv_rn(__uint_as_float(u[2 * e + 1] << 16), s);
+                const float v3 = __fdiv_rn(__uint_as_float(u[2 * e + 1] & 0xFFFF0000u), s);
+                out[e] = e4m3x2(v0, v1) | (e4m3x2(v2, v3) << 16);
             }
             dst[i] = make_uint4(out[0], out[1], out[2], out[3]);
         }
@@ -135,9 +167,12 @@ int check_arch()
     return DIT_ATTN_OK;
 }
 
-int grid_rows(long long rows)
+// Grid of a row-chunked kernel: chunks of `per_cta` units per row in x, rows
+// in y (capped; the kernels stride over the remaining rows).
+dim3 grid_rows(long long rows, long long units_per_row, long long per_cta)
 {
-    return (int)(rows < 148ll * 8 ? rows : 148ll * 8);
+    const long long chunks = (units_per_row + per_cta - 1) / per_cta;
+    return dim3((unsigned)chunks, (unsigned)(rows < 65535 ? rows : 65535));
 }
 
 } // namespace
@@ -185,8 +220,10 @@ extern "C" int dit_attn_absmax_rows(const void *x, float *amax, long long rows, 
     const int rc = check_arch();
     if (rc != DIT_ATTN_OK)
         return rc;
-    absmax_rows_kernel<<<grid_rows(rows), kThreads, 0, stream>>>(static_cast<const uint4 *>(x), amax, rows,
-                                                                 row_len / 8);
+    if (cudaMemsetAsync(amax, 0, (size_t)rows * sizeof(float), stream) != cudaSuccess)
+        return DIT_ATTN_ERR_LAUNCH;
+    absmax_rows_kernel<<<grid_rows(rows, row_len / 8, kUnitsPerCta), kThreads, 0, stream>>>(
+        static_cast<const uint4 *>(x), reinterpret_cast<unsigned int *>(amax), rows, row_len / 8);
     return cudaGetLastError() == cudaSuccess ? DIT_ATTN_OK : DIT_ATTN_ERR_LAUNCH;
 }
 
@@ -204,8 +241,7 @@ extern "C" int dit_attn_quantize_e4m3_rows(const void *x, const float *amax, voi
     const int rc = check_arch();
     if (rc != DIT_ATTN_OK)
         return rc;
-    quantize_rows_kernel<<<grid_rows(rows), kThreads, 0, stream>>>(static_cast<const uint4 *>(x),
-                                                                   static_cast<uint4 *>(q), amax, scale_out, rows,
-                                                                   row_len / 16);
+    quantize_rows_kernel<<<grid_rows(rows, row_len / 16, kUnitsPerCta), kThreads, 0, stream>>>(
+        static_cast<const uint4 *>(x), static_cast<uint4 *>(q), amax, scale_out, rows, row_len / 16);
     return cudaGetLastError() == cudaSuccess ? DIT_ATTN_OK : DIT_ATTN_ERR_LAUNCH;
 }

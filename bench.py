@@ -26,6 +26,10 @@ hot path is one kernel launch).  Prints ONE JSON line on rank 0.
   the previous step's); GB/s of algorithmic HBM traffic.
 * --op mxfp4_quant: the MXFP4 1x32 activation quantiser on a (B*L) x (H*D)
   bf16 activation of the workload; GB/s of algorithmic HBM traffic.
+* --op ulysses_fp8_payload: the per-GPU preparation of Ulysses' FP8 all-to-all
+  payload for one [B, H, L, D] bf16 tensor of the workload: per-head absmax,
+  e4m3 quantisation, heads grouped by destination rank; GB/s of algorithmic
+  HBM traffic (roofline: the quantiser, the step's largest kernel).
 Multi-GPU (torchrun): every rank runs its own replica (no data exchange:
 heads and batches are independent), scaling "weak".
 """
@@ -49,6 +53,8 @@ METRIC = "attention TFLOP/s and % of B200 tensor-core peak at 1 GPU"
 MERGE_METRIC = "LSE merge of partial attentions: GB/s of algorithmic HBM traffic at 1 GPU"
 DIFF_METRIC = "step-cache residual-change decision: GB/s of algorithmic HBM traffic at 1 GPU"
 MXFP4_METRIC = "MXFP4 1x32 activation quantiser: GB/s of algorithmic HBM traffic at 1 GPU"
+PAYLOAD_METRIC = ("Ulysses FP8 payload preparation (absmax, e4m3 quantise, head grouping): "
+                  "GB/s of algorithmic HBM traffic at 1 GPU")
 DEFAULT_WORKLOAD = "flux_2048_cfg"      # the first workload with L >= 16k (the stated target)
 NOMINAL_TFLOPS = {"bf16": 2250.0, "e4m3": 4500.0}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
@@ -73,6 +79,7 @@ KERNEL_SOURCES = {
     "lse_merge": ["lse_merge.cu"],
     "residual_diff": ["residual_diff.cu"],
     "mxfp4_quant": ["mxfp4_quant.cu"],
+    "ulysses_ops": ["ulysses_ops.cu"],
 }
 
 
@@ -802,6 +809,197 @@ def run_mxfp4(args, dist: Dist):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ Ulysses FP8 payload
+
+def ulysses_degree(H: int) -> int:
+    """The largest of 8, 4, 2, 1 ranks that the heads split over evenly."""
+    return next(n for n in (8, 4, 2, 1) if H % n == 0)
+
+
+def payload_bytes(n: int, rows: int) -> int:
+    """absmax reads 2n bytes and writes the row maxima; the quantiser reads 2n
+    and the maxima, writes n and the scales; the head grouping reads and
+    writes n."""
+    return 7 * n + 12 * rows
+
+
+def payload_config(w, N):
+    n = w.B * w.H * w.L * w.D
+    return {"workload": w.name, "op": "ulysses_fp8_payload", "shape": [w.B, w.H, w.L, w.D],
+            "ranks": N, "input_dtype": "bf16", "payload": "e4m3 + fp32 per-head scales",
+            "bytes_per_call": payload_bytes(n, w.B * w.H),
+            "kernels": ["absmax_rows_kernel", "quantize_rows_kernel", "block_transpose_kernel"],
+            "note": "one rank's tensor; the all-reduce of the head maxima and the all-to-all are "
+                    "collectives across GPUs, not part of this single-GPU step",
+            "l2": "inputs larger than L2" if 2 * n > L2_BYTES else "L2 flushed between timed steps (256 MB write)",
+            "parallelism": "replicas"}
+
+
+def payload_oracle_rate(x_cpu, rows: int, N: int, B: int, seconds: float):
+    """Oracle rate over whole heads (rows) of x_cpu [rows, row_len], as many as
+    fit in about seconds/4 (the head grouping over the quantised sample)."""
+    from oracle import e4m3_payload as ep
+    r = 1
+    while True:
+        xs = x_cpu[:r].double().numpy()
+        t0 = time.perf_counter()
+        amax = ep.absmax_rows(xs, r)
+        qc, _ = ep.quantize_rows(xs, amax)
+        if r % N == 0:
+            ep.block_transpose(qc, r // N, N)
+        dt = time.perf_counter() - t0
+        if dt >= seconds / 4 or r >= rows:
+            return payload_bytes(xs.size, r) / dt / 1e9, r, dt
+        r = min(rows, r * 2)
+
+
+def payload_input(w, dev):
+    import torch
+    g = torch.Generator(device=dev).manual_seed(w.seed)
+    return torch.randn((w.B, w.H, w.L, w.D), generator=g, device=dev).to(torch.bfloat16)
+
+
+def run_payload_reference(args, dist: Dist):
+    if dist.rank != 0:
+        return
+    import torch
+    from attention_dit_attn_b200 import workloads as wl
+    w = wl.ALL[args.workload]
+    N = ulysses_degree(w.H)
+    rows, row_len = w.B * w.H, w.L * w.D
+    g = torch.Generator().manual_seed(w.seed)
+    x = torch.randn((min(rows, 8), row_len), generator=g).to(torch.bfloat16)
+    per = 60.0 / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        payload_oracle_rate(x, x.shape[0], N, w.B, per)
+    rates = [payload_oracle_rate(x, x.shape[0], N, w.B, per) for _ in range(args.steps)]
+    value = statistics.median(r[0] for r in rates)
+    nbytes = payload_bytes(rows * row_len, rows)
+    line = {
+        "impl": "reference", "metric": PAYLOAD_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * nbytes / (value * 1e9),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": payload_config(w, N),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: fp64 numpy oracle on {rates[0][1]} head(s) of {row_len} values"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_payload(args, dist: Dist):
+    import torch
+    import attention_dit_attn_b200 as dit
+    from attention_dit_attn_b200 import workloads as wl
+
+    dit.ensure_built()
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    w = wl.ALL[args.workload]
+    N = ulysses_degree(w.H)
+    rows = w.B * w.H
+    x = payload_input(w, dev)
+    n = x.numel()
+    amax = torch.empty(rows, dtype=torch.float32, device=dev)
+    q8 = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=dev)
+    sc = torch.empty(rows, dtype=torch.float32, device=dev)
+    out = torch.empty_like(q8)
+    nbytes = payload_bytes(n, rows)
+    flush = None
+    if 2 * n <= L2_BYTES:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xx, evq=None):
+        dit.dit_attn_absmax_rows(xx, rows, amax, stream=stream)
+        if evq is not None:
+            evq[0].record(stream)
+        dit.dit_attn_quantize_e4m3_rows(xx, amax, q8, sc, stream=stream)
+        if evq is not None:
+            evq[1].record(stream)
+        dit.dit_attn_block_transpose(q8, w.B, N, out, stream=stream)   # [B, N, H/N, ...] -> [N, B, H/N, ...]
+
+    for _ in range(args.warmup):
+        step(x)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler()
+    if dist.rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    evs = [(ev(), ev(), (ev(), ev())) for _ in range(args.steps)]
+    for a, b, evq in evs:
+        if flush is not None:
+            flush.fill_(1)
+        a.record(stream)
+        step(x, evq)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    seconds = sum(a.elapsed_time(b) for a, b, _ in evs) / 1e3
+    q_seconds = sum(e0.elapsed_time(e1) for _, _, (e0, e1) in evs) / 1e3
+    dist.barrier()
+    if dist.rank == 0:
+        time.sleep(0.2)
+        sampler.stop()
+    max_seconds = dist.max(seconds, dev)
+    value = nbytes * args.steps * dist.world / max_seconds / 1e9
+    q_bytes = 3 * n + 4 * rows + 4 * rows
+    achieved = q_bytes / (q_seconds / args.steps) / 1e9
+
+    e2e_steps = max(3, min(args.steps, 10))
+    hx = x.cpu().pin_memory()
+    dx = torch.empty_like(x)
+    hout = torch.empty(out.shape, dtype=torch.uint8).pin_memory()
+    hs = torch.empty(sc.shape, dtype=sc.dtype).pin_memory()
+
+    def e2e_step():
+        dx.copy_(hx, non_blocking=True)
+        step(dx)
+        hout.copy_(out.view(torch.uint8), non_blocking=True)
+        hs.copy_(sc, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    a, b = ev(), ev()
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = dist.max(a.elapsed_time(b) / 1e3, dev)
+
+    peaks, peaks_kind = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    traffic = profiled_traffic(w.name, kind="ulysses_ops")
+    clocks = sampler.summary(physical_gpu_index(dist.local_rank)) if dist.rank == 0 else {}
+    line = {
+        "metric": PAYLOAD_METRIC, "value": value, "unit": "GB/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * max_seconds / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": payload_config(w, N),
+        "e2e": {"value": nbytes * e2e_steps * dist.world / e2e_s / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": 2 * n, "d2h_bytes_per_step": n + 4 * rows,
+                "steps": e2e_steps,
+                "result_matches_device": bool(torch.equal(hout, out.view(torch.uint8).cpu()) and torch.equal(hs, sc.cpu()))},
+        "gpu_launches": 3 * args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"HBM copy, {peaks_kind}", "traffic": traffic,
+                     "kernel": "quantize_rows_kernel", "bytes_per_launch": q_bytes},
+        "clocks": clocks,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        xr = x.reshape(rows, -1)[:8].cpu()
+        rate, sr, dt = payload_oracle_rate(xr, xr.shape[0], N, w.B, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": f"fp64 numpy oracle on the first {sr} head(s) of {xr.shape[1]} values: {dt:.2f} s"}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, dist: Dist):
     import torch
     import attention_dit_attn_b200 as dit
@@ -951,7 +1149,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["attention", "lse_merge", "residual_diff", "mxfp4_quant"], default="attention")
+    ap.add_argument("--op", choices=["attention", "lse_merge", "residual_diff", "mxfp4_quant", "ulysses_fp8_payload"],
+                    default="attention")
     ap.add_argument("--parts", type=int, default=2, help="lse_merge: number of partial results (ring degree)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -965,12 +1164,13 @@ def main(argv=None):
         # The oracle runs on rank 0's host cores only; other ranks exit at once.
         if int(os.environ.get("RANK", "0")) == 0:
             {"lse_merge": run_merge_reference, "residual_diff": run_diff_reference,
-             "mxfp4_quant": run_mxfp4_reference}.get(
+             "mxfp4_quant": run_mxfp4_reference, "ulysses_fp8_payload": run_payload_reference}.get(
                 args.op, run_reference)(args, Dist.single())
         return
     dist = Dist(args.gpus)
     try:
-        {"lse_merge": run_merge, "residual_diff": run_diff, "mxfp4_quant": run_mxfp4}.get(
+        {"lse_merge": run_merge, "residual_diff": run_diff, "mxfp4_quant": run_mxfp4,
+         "ulysses_fp8_payload": run_payload}.get(
             args.op, run_ours)(args, dist)
     finally:
         dist.close()

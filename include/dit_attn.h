@@ -261,7 +261,10 @@ int dit_attn_block_transpose(const void *in, void *out, long long R, long long C
 /*
  * dit_attn_absmax_rows — amax[r] = max_i |x[r][i]| (fp32) for bf16 rows of
  * row_len values (a multiple of 8), e.g. rows = B*H of a [B, H, Ls, D] shard.
- * x 16-byte aligned.  rows = 0: nothing is enqueued.
+ * x 16-byte aligned, amax 4-byte aligned.  Enqueues a zero fill of amax and
+ * one kernel whose CTAs each take a chunk of a row and combine their maxima
+ * atomically (the result does not depend on their order).  rows = 0: nothing
+ * is enqueued.
  */
 int dit_attn_absmax_rows(const void *x, float *amax, long long rows, long long row_len, cudaStream_t stream);
 

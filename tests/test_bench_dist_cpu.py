@@ -78,7 +78,8 @@ def test_bench_rejects_too_few_warmup_steps():
     assert r.returncode != 0
 
 
-@pytest.mark.parametrize("op,unit", [("lse_merge", "GB/s"), ("residual_diff", "GB/s"), ("mxfp4_quant", "GB/s")])
+@pytest.mark.parametrize("op,unit", [("lse_merge", "GB/s"), ("residual_diff", "GB/s"), ("mxfp4_quant", "GB/s"),
+                                     ("ulysses_fp8_payload", "GB/s")])
 def test_reference_arm_of_each_op_prints_one_json_line(op, unit):
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--op", op, "--workload", "tiny_256",
                         "--steps", "3", "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=300)
@@ -89,3 +90,10 @@ def test_reference_arm_of_each_op_prints_one_json_line(op, unit):
     assert d["impl"] == "reference" and d["unit"] == unit and d["value"] > 0
     assert d["config"]["op"] == op and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_payload_byte_count_and_ulysses_degree():
+    import bench
+    assert [bench.ulysses_degree(h) for h in (24, 38, 40, 2, 3)] == [8, 2, 8, 2, 1]
+    # absmax 2n + quantiser 3n + head grouping 2n, plus 12 bytes per row of maxima and scales.
+    assert bench.payload_bytes(1000, 4) == 7000 + 48
