@@ -1076,34 +1076,58 @@ def run_ours(args, dist: Dist):
     kernel_avg_s = kernel_ms_total / 1e3 / args.steps
     launches = args.steps * dit.dit_attn_launches_per_call(w.B, w.H, w.L, w.D, 0 if w.dtype == "bf16" else 1)
 
-    # ---- end to end through the public API, host buffers, copies in the timed region
+    # ---- end to end through the public API, host buffers, copies in the timed region.
+    # Every step copies its q/k/v in from pinned host memory and its o/lse back
+    # out.  Two device buffer sets and three streams let the copies of one step
+    # overlap the attention of the neighbouring step, as a serving loop would.
     e2e_steps = max(3, min(args.steps, 10))
     hq, hk, hv = (t.pin_memory() for t in (inp.q, inp.k, inp.v))
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    bufs = [dict(q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v), o=torch.empty_like(o),
+                 lse=torch.empty_like(lse)) for _ in range(2)]
+    s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    in_done, cmp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        dit.dit_attn_fwd(dq, dk, dv, o, lse, scale=w.scale, stream=stream, **kw)
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
+    def e2e_run(n_steps, start=None, end=None):
+        if start is not None:
+            start.record(s_in)
+        for i in range(n_steps):
+            b = i % 2
+            buf = bufs[b]
+            if i >= 2:
+                s_in.wait_event(cmp_done[b])         # step i-2's attention has read this buffer set
+            with torch.cuda.stream(s_in):
+                buf["q"].copy_(hq, non_blocking=True)
+                buf["k"].copy_(hk, non_blocking=True)
+                buf["v"].copy_(hv, non_blocking=True)
+            in_done[b].record(s_in)
+            s_cmp.wait_event(in_done[b])
+            if i >= 2:
+                s_cmp.wait_event(out_done[b])        # step i-2's o/lse have been copied out
+            dit.dit_attn_fwd(buf["q"], buf["k"], buf["v"], buf["o"], buf["lse"], scale=w.scale, stream=s_cmp,
+                             **kw)
+            cmp_done[b].record(s_cmp)
+            s_out.wait_event(cmp_done[b])
+            with torch.cuda.stream(s_out):
+                ho.copy_(buf["o"], non_blocking=True)
+                hl.copy_(buf["lse"], non_blocking=True)
+            out_done[b].record(s_out)
+        if end is not None:
+            end.record(s_out)
 
-    e2e_step()
+    e2e_run(2)
     torch.cuda.synchronize(dev)
     dist.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    b.record(stream)
+    e2e_run(e2e_steps, a, b)
     torch.cuda.synchronize(dev)
     e2e_s = dist.max(a.elapsed_time(b) / 1e3, dev)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
-    e2e_ok = torch.equal(ho, o.cpu())
+    last = bufs[(e2e_steps - 1) % 2]
+    e2e_ok = bool(torch.equal(ho, last["o"].cpu()) and torch.equal(hl, last["lse"].cpu()) and torch.equal(ho, o.cpu()))
 
     peaks, peaks_kind = load_peaks()
     if w.dtype == "bf16":
