@@ -27,7 +27,8 @@ __all__ = [
     "dit_attn_lse_merge_ptr", "DIT_ATTN_MERGE_MAX_PARTS", "dit_attn_residual_diff",
     "dit_attn_residual_diff_ptr", "dit_attn_residual_diff_workspace_bytes", "dit_attn_residual_diff_noalloc",
     "dit_attn_mxfp4_quantize", "dit_attn_mxfp4_quantize_ptr", "dit_attn_block_transpose",
-    "dit_attn_absmax_rows", "dit_attn_quantize_e4m3_rows",
+    "dit_attn_absmax_rows", "dit_attn_quantize_e4m3_rows", "dit_attn_fwd_ulysses", "dit_attn_fwd_ulysses_ptr",
+    "dit_attn_ulysses_check_device_error",
     "ensure_built", "lib",
     "header_functions", "STATUS",
 ]
@@ -97,6 +98,11 @@ def lib() -> ctypes.CDLL:
         L.dit_attn_lse_merge.restype = i32
         L.dit_attn_lse_merge.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i32, vp, vp,
                                          ctypes.c_longlong, i32, vp]
+        L.dit_attn_fwd_ulysses.restype = i32
+        L.dit_attn_fwd_ulysses.argtypes = [ctypes.POINTER(vp)] * 5 + [i32] * 6 + [ctypes.c_float, i32, vp, vp, vp,
+                                                                                vp]
+        L.dit_attn_ulysses_check_device_error.restype = i32
+        L.dit_attn_ulysses_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         _lib = L
     return _lib
 
@@ -383,3 +389,64 @@ def dit_attn_quantize_e4m3_rows(x, amax, q=None, scale=None, *, stream=None):
                                              x.numel() // max(rows, 1), _stream_handle(stream)),
            "dit_attn_quantize_e4m3_rows")
     return q, scale
+
+
+def dit_attn_fwd_ulysses_ptr(q: list[int], k: list[int], v: list[int], o: list[int], lse: list[int] | None,
+                             rank: int, B: int, H: int, Ls: int, D: int, scale: float, dtype: int,
+                             q_scale: int | None = None, k_scale: int | None = None, v_scale: int | None = None,
+                             stream: int = 0) -> int:
+    """Raw C-ABI call: per-shard integer device pointers (lists of n_ranks); returns the status."""
+    n = len(q)
+    arr = lambda xs: (ctypes.c_void_p * max(n, 1))(*[ctypes.c_void_p(x) for x in xs])
+    return lib().dit_attn_fwd_ulysses(arr(q), arr(k), arr(v), arr(o), None if lse is None else arr(lse), n, rank,
+                                      B, H, Ls, D, ctypes.c_float(scale), dtype, q_scale, k_scale, v_scale, stream)
+
+
+def dit_attn_fwd_ulysses(q_shards, k_shards, v_shards, o_shards, lse_shards=None, *, rank: int,
+                         scale: float | None = None, q_scale=None, k_scale=None, v_scale=None, stream=None):
+    """Ulysses attention with the exchanges fused into the kernel.  Shard c of each
+    list is a contiguous CUDA tensor [B, H, Ls, D] holding tokens c*Ls .. c*Ls + Ls of
+    all heads (q/k/v bf16, or float8_e4m3fn with [B, H] fp32 scales of all heads; o bf16;
+    lse fp32 [B, H, Ls] or None).  Computes attention over all n*Ls tokens for head group
+    `rank` (H/n heads) and writes those heads' rows of every o/lse shard.  The tensors may
+    live on other GPUs if their memory is mapped into this context."""
+    import torch
+    n = len(q_shards)
+    if not (len(k_shards) == len(v_shards) == len(o_shards) == n) or (lse_shards is not None and len(lse_shards) != n):
+        raise ValueError("one shard of each tensor per rank")
+    B, H, Ls, D = q_shards[0].shape
+    for t in (*q_shards, *k_shards, *v_shards):
+        if t.shape != (B, H, Ls, D) or t.dtype != q_shards[0].dtype or not t.is_contiguous():
+            raise ValueError("q/k/v shards must be contiguous [B, H, Ls, D] tensors of one dtype")
+    for t in o_shards:
+        if t.shape != (B, H, Ls, D) or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("o shards must be contiguous bf16 [B, H, Ls, D] tensors")
+    if lse_shards is not None:
+        for t in lse_shards:
+            if t.numel() != B * H * Ls or t.dtype != torch.float32 or not t.is_contiguous():
+                raise ValueError("lse shards must be contiguous fp32 tensors of B*H*Ls elements")
+    if q_shards[0].dtype == torch.bfloat16:
+        dtype, scales = DIT_ATTN_BF16, (None, None, None)
+    elif q_shards[0].dtype == torch.float8_e4m3fn:
+        dtype = DIT_ATTN_FP8_E4M3
+        scales = []
+        for name, s in (("q_scale", q_scale), ("k_scale", k_scale), ("v_scale", v_scale)):
+            if s is None or not s.is_cuda or s.dtype != torch.float32 or s.numel() != B * H or not s.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor with B*H elements")
+            scales.append(s.data_ptr())
+    else:
+        raise TypeError(f"unsupported dtype {q_shards[0].dtype}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    ptrs = lambda ts: [t.data_ptr() for t in ts]
+    rc = dit_attn_fwd_ulysses_ptr(ptrs(q_shards), ptrs(k_shards), ptrs(v_shards), ptrs(o_shards),
+                                  None if lse_shards is None else ptrs(lse_shards), rank, B, H, Ls, D, float(scale),
+                                  dtype, *scales, stream=_stream_handle(stream))
+    _check(rc, "dit_attn_fwd_ulysses")
+
+
+def dit_attn_ulysses_check_device_error(stream=None) -> tuple[int, int]:
+    """The fused Ulysses kernel's device error word: synchronise, read, clear: (status, raw word)."""
+    word = ctypes.c_uint32(0)
+    rc = lib().dit_attn_ulysses_check_device_error(_stream_handle(stream), ctypes.byref(word))
+    return rc, word.value

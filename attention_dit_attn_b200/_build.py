@@ -10,8 +10,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdit_attn.so")
-SOURCES = ["dit_attn.cu", "lse_merge.cu", "residual_diff.cu", "mxfp4_quant.cu", "ulysses_ops.cu"]
-DEPS = ["dit_attn.cu", "lse_merge.cu", "residual_diff.cu", "mxfp4_quant.cu", "ulysses_ops.cu", "attn_common.cuh", "attn_fwd_sm100.cuh", "sm100_ptx.cuh"]
+SOURCES = ["dit_attn.cu", "lse_merge.cu", "residual_diff.cu", "mxfp4_quant.cu", "ulysses_ops.cu", "ulysses_fused.cu"]
+DEPS = ["dit_attn.cu", "lse_merge.cu", "residual_diff.cu", "mxfp4_quant.cu", "ulysses_ops.cu", "ulysses_fused.cu",
+        "attn_common.cuh", "attn_fwd_sm100.cuh", "attn_fwd_ulysses_sm100.cuh", "sm100_ptx.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

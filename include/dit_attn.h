@@ -280,6 +280,50 @@ int dit_attn_quantize_e4m3_rows(const void *x, const float *amax, void *q, float
                                 long long row_len, cudaStream_t stream);
 
 /*
+ * dit_attn_fwd_ulysses — Ulysses attention with both exchanges fused into
+ * the attention kernel (page "How to Scale Diffusion Inference Across AMD
+ * RDNA 4 GPUs", section "Balance Transformer Work and Communication").
+ *
+ * n_ranks shards, shard c holding tokens [c Ls, (c + 1) Ls) of the joint
+ * sequence for all H heads: q_shards[c], k_shards[c], v_shards[c] are
+ * [B, H, Ls, D] (bf16, or e4m3 with dtype DIT_ATTN_FP8_E4M3), o_shards[c]
+ * [B, H, Ls, D] bf16, lse_shards[c] [B, H, Ls] fp32.  The call computes
+ * dit_attn_fwd's attention over all L = n_ranks Ls tokens for the head group
+ * [rank H / n_ranks, (rank + 1) H / n_ranks), reading every tile from the
+ * shard that holds it, and writes those heads' rows of every shard's O and
+ * LSE; other heads' rows are not touched.  The n_ranks calls rank = 0 ..
+ * n_ranks - 1 together produce the whole attention in the shards' layout.
+ *
+ * The pointer arrays are host arrays of n_ranks device pointers.  A pointer
+ * may address another GPU's memory mapped into the current context (CUDA IPC
+ * or peer access, set up by the caller); the kernel reads and writes it with
+ * plain TMA copies (no cluster multicast).  The caller orders the call after
+ * every shard's q/k/v are written and orders readers of o/lse after the calls
+ * of all ranks that write them (on several GPUs: a stream synchronisation and
+ * a barrier of the process group).
+ *
+ * FP8: q/k/v_scale are [B, H] dequantisation scales of all heads, the same in
+ * every shard (per-head scales agreed across ranks).  lse_shards may be NULL
+ * (no LSE); otherwise every entry is non-NULL.
+ * Requirements: 1 <= n_ranks <= 8, 0 <= rank < n_ranks, H % n_ranks == 0,
+ * Ls % 64 == 0, D in {64, 128}, every pointer 16-byte aligned (LSE 4-byte).
+ * Errors as dit_attn_fwd (before anything is enqueued).  Device-side wait
+ * timeouts (4 s) are reported by dit_attn_ulysses_check_device_error.
+ */
+int dit_attn_fwd_ulysses(const void *const *q_shards, const void *const *k_shards, const void *const *v_shards,
+                         void *const *o_shards, float *const *lse_shards, int n_ranks, int rank, int B, int H,
+                         int Ls, int D, float scale, int dtype, const float *q_scale, const float *k_scale,
+                         const float *v_scale, cudaStream_t stream);
+
+/*
+ * dit_attn_ulysses_check_device_error — dit_attn_check_device_error for the
+ * fused Ulysses kernel (it keeps its own device error word): synchronises
+ * `stream`, returns DIT_ATTN_ERR_TIMEOUT (and clears the word) if a wait of
+ * that kernel timed out, with the word in *detail if detail is non-NULL.
+ */
+int dit_attn_ulysses_check_device_error(cudaStream_t stream, uint32_t *detail);
+
+/*
  * dit_attn_residual_diff_noalloc — dit_attn_residual_diff without a caller
  * workspace and without allocating anything: the scratch is a fixed array in
  * the library's own device memory (zero at load, left zero by every call),

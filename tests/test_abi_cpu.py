@@ -21,7 +21,8 @@ def test_library_exports_every_header_function(L):
                           "dit_attn_launches_per_call", "dit_attn_lse_merge", "dit_attn_residual_diff",
                           "dit_attn_residual_diff_workspace_bytes", "dit_attn_residual_diff_noalloc",
                           "dit_attn_mxfp4_quantize", "dit_attn_block_transpose", "dit_attn_absmax_rows",
-                          "dit_attn_quantize_e4m3_rows"}
+                          "dit_attn_quantize_e4m3_rows", "dit_attn_fwd_ulysses",
+                          "dit_attn_ulysses_check_device_error"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -162,3 +163,19 @@ def test_ulysses_ops_argument_validation(L):
     assert L.dit_attn_quantize_e4m3_rows(16, 16, 16, None, 4, 24, None) == 2   # row_len not a multiple of 16
     assert L.dit_attn_quantize_e4m3_rows(16, 16, None, None, 4, 64, None) == 1
     assert L.dit_attn_quantize_e4m3_rows(16, 16, 16, None, 4, 64, None) == 5
+
+
+def test_fused_ulysses_argument_validation(L):
+    call = dit.dit_attn_fwd_ulysses_ptr
+    two = [16, 16]
+    assert call([16], [16], [16], [16], None, 0, 1, 1, 64, 64, 0.1, 0) == 5       # well-formed: no GPU here
+    assert call(two, two, two, two, None, 0, 1, 3, 64, 64, 0.1, 0) == 2          # H % n_ranks
+    assert call(two, two, two, two, None, 0, 1, 4, 100, 64, 0.1, 0) == 2         # Ls % 64
+    assert call(two, two, two, two, None, 2, 1, 4, 64, 64, 0.1, 0) == 2          # rank out of range
+    assert call([16] * 9, [16] * 9, [16] * 9, [16] * 9, None, 0, 1, 9, 64, 64, 0.1, 0) == 2   # > 8 ranks
+    assert call(two, two, two, [16, 0], None, 0, 1, 4, 64, 64, 0.1, 0) == 1      # a NULL shard
+    assert call(two, two, two, two, [16, 0], 0, 1, 4, 64, 64, 0.1, 0) == 1       # LSE for some shards only
+    assert call(two, two, [16, 24], two, None, 0, 1, 4, 64, 64, 0.1, 0) == 4     # misaligned shard
+    assert call(two, two, two, two, None, 0, 1, 4, 64, 96, 0.1, 0) == 2          # head dim
+    assert call(two, two, two, two, None, 0, 1, 4, 64, 64, 0.1, 1) == 1          # FP8 without scales
+    assert call(two, two, two, two, None, 0, 1, 4, 64, 64, -1.0, 0) == 8         # negative scale
