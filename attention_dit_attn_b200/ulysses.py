@@ -20,6 +20,11 @@ The exchange is torch.distributed (NCCL between GPUs).  The per-GPU steps go
 through ``ops``: by default this library's kernels (dit_attn_block_transpose,
 dit_attn_absmax_rows, dit_attn_quantize_e4m3_rows, dit_attn_fwd); tests on CPU
 pass reference ops to check the exchange logic with gloo ranks.
+
+dit_attn_fwd_ulysses is the fused alternative: given every rank's shard
+pointers (peers' memory mapped into this context), one kernel per rank reads
+the tiles from the shards and writes O and the LSE back into them, with no
+all-to-all and no gathered copy.
 """
 from __future__ import annotations
 
