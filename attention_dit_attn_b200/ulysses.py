@@ -102,3 +102,38 @@ def ulysses_attention(q, k, v, *, group=None, scale: float | None = None, fp8_co
     l_recv = _all_to_all(ops.block_transpose(lse.contiguous(), B * Hn, N), group)
     l_out = ops.block_transpose(l_recv, N, B).view(B, H, Ls)
     return o_out, l_out
+
+
+def ulysses_attention_fused(q, k, v, *, group=None, scale: float | None = None, q_scale=None, k_scale=None,
+                            v_scale=None):
+    """The fused path of ulysses_attention: the same inputs (this rank's shard
+    [B, H, Ls, D] of q, k, v; FP8 with [B, H] per-head scales agreed by all ranks)
+    and the same result (this rank's shard of O and the LSE over the whole
+    sequence), computed by dit_attn_fwd_ulysses with every rank's shards mapped
+    into this process through CUDA IPC.  All ranks of ``group`` run on one node;
+    ``group`` may be any backend (it carries only the IPC handles and barriers).
+    Ls must be a multiple of 64 and H a multiple of the group size."""
+    import torch
+    import torch.distributed as dist
+    from torch.multiprocessing.reductions import reduce_tensor
+
+    from . import dit_attn_fwd_ulysses
+    N = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    B, H, Ls, D = q.shape
+    o = torch.empty((B, H, Ls, D), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, Ls), dtype=torch.float32, device=q.device)
+    local = [t.contiguous() for t in (q, k, v)] + [o, lse]
+    handles = [None] * N
+    dist.all_gather_object(handles, [reduce_tensor(t) for t in local], group=group)
+    shards = [local if c == rank else [fn(*args) for fn, args in handles[c]] for c in range(N)]
+    torch.cuda.synchronize(q.device)
+    dist.barrier(group=group)            # every rank's q/k/v are written and mapped
+    dit_attn_fwd_ulysses([s[0] for s in shards], [s[1] for s in shards], [s[2] for s in shards],
+                         [s[3] for s in shards], [s[4] for s in shards], rank=rank, scale=scale,
+                         q_scale=q_scale, k_scale=k_scale, v_scale=v_scale)
+    torch.cuda.synchronize(q.device)
+    dist.barrier(group=group)            # every rank's writes into this rank's o/lse are done
+    del shards, handles
+    dist.barrier(group=group)            # no rank still maps another's memory
+    return o, lse
