@@ -98,3 +98,13 @@ def test_block_transpose_by_hand():
     out = ep.block_transpose(b, 2, 3)
     assert list(out) == [0, 1, 6, 7, 2, 3, 8, 9, 4, 5, 10, 11]
     assert np.array_equal(ep.block_transpose(out, 3, 2), b)
+
+
+def test_block_transpose_and_absmax_agree_with_the_torch_reference_ops():
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn((2, 6, 40, 16), generator=g).to(torch.bfloat16)
+    ref = RefOps()
+    got = ep.block_transpose(x.view(torch.int16).numpy(), 2, 3)
+    want = ref.block_transpose(x, 2, 3).contiguous().view(torch.uint8).numpy().reshape(-1)
+    assert np.array_equal(got, want)
+    assert np.array_equal(ep.absmax_rows(x.double().numpy(), 12), ref.absmax_rows(x, 12).double().numpy())
