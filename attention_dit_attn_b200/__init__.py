@@ -286,6 +286,8 @@ def dit_attn_residual_diff(cur, prev, threshold: float = 0.12, *, workspace=None
         diff = torch.empty(1, dtype=torch.float32, device=cur.device)
     if reuse is None:
         reuse = torch.empty(1, dtype=torch.int32, device=cur.device)
+    _require(diff, "diff", (torch.float32,), 1)
+    _require(reuse, "reuse", (torch.int32,), 1)
     rc = dit_attn_residual_diff_ptr(cur.data_ptr(), prev.data_ptr(), n, float(threshold), workspace.data_ptr(),
                                     workspace.numel(), diff.data_ptr(), reuse.data_ptr(), _stream_handle(stream))
     if rc != 0:
@@ -307,6 +309,8 @@ def dit_attn_residual_diff_noalloc(cur, prev, threshold: float = 0.12, *, diff=N
         diff = torch.empty(1, dtype=torch.float32, device=cur.device)
     if reuse is None:
         reuse = torch.empty(1, dtype=torch.int32, device=cur.device)
+    _require(diff, "diff", (torch.float32,), 1)
+    _require(reuse, "reuse", (torch.int32,), 1)
     rc = lib().dit_attn_residual_diff_noalloc(cur.data_ptr(), prev.data_ptr(), cur.numel(), ctypes.c_float(threshold),
                                               diff.data_ptr(), reuse.data_ptr(), _stream_handle(stream))
     if rc != 0:
@@ -346,6 +350,21 @@ def _check(rc: int, what: str):
         raise DitAttnError(rc, what + ": ")
 
 
+def _require(t, name: str, dtypes=None, numel: int | None = None, nbytes: int | None = None):
+    """A caller-provided tensor must be a contiguous CUDA tensor (a host pointer reaching
+    a kernel would fault), of one of `dtypes`, with `numel` elements or `nbytes` bytes."""
+    import torch
+    ok = isinstance(t, torch.Tensor) and t.is_cuda and t.is_contiguous()
+    ok = ok and (dtypes is None or t.dtype in dtypes)
+    ok = ok and (numel is None or t.numel() == numel)
+    ok = ok and (nbytes is None or t.numel() * t.element_size() == nbytes)
+    if not ok:
+        want = "" if dtypes is None else " of dtype " + "/".join(str(d) for d in dtypes)
+        size = "" if numel is None else f" with {numel} elements"
+        size += "" if nbytes is None else f" of {nbytes} bytes"
+        raise ValueError(f"{name} must be a contiguous CUDA tensor{want}{size}")
+
+
 def dit_attn_block_transpose(x, R: int, C: int, out=None, *, stream=None):
     """out[c][r] = x[r][c] over an R x C grid of equal contiguous blocks of a CUDA tensor
     (its bytes split into R*C blocks).  Returns a tensor of x's dtype and numel."""
@@ -357,6 +376,7 @@ def dit_attn_block_transpose(x, R: int, C: int, out=None, *, stream=None):
         raise ValueError("x's bytes must split into R*C equal blocks")
     if out is None:
         out = torch.empty_like(x)
+    _require(out, "out", nbytes=nbytes)
     _check(lib().dit_attn_block_transpose(x.data_ptr(), out.data_ptr(), R, C, nbytes // (R * C),
                                           _stream_handle(stream)), "dit_attn_block_transpose")
     return out
@@ -367,8 +387,11 @@ def dit_attn_absmax_rows(x, rows: int, out=None, *, stream=None):
     import torch
     if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous()):
         raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    if rows < 0 or (rows == 0 and x.numel()) or (rows > 0 and x.numel() % rows):
+        raise ValueError("x must split into `rows` equal rows")
     if out is None:
         out = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _require(out, "out", (torch.float32,), rows)
     _check(lib().dit_attn_absmax_rows(x.data_ptr(), out.data_ptr(), rows, x.numel() // max(rows, 1),
                                       _stream_handle(stream)), "dit_attn_absmax_rows")
     return out
@@ -380,11 +403,16 @@ def dit_attn_quantize_e4m3_rows(x, amax, q=None, scale=None, *, stream=None):
     import torch
     if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous()):
         raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    _require(amax, "amax", (torch.float32,))
     rows = amax.numel()
+    if (rows == 0 and x.numel()) or (rows > 0 and x.numel() % rows):
+        raise ValueError("x must split into amax.numel() equal rows")
     if q is None:
         q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
     if scale is None:
         scale = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _require(q, "q", (torch.float8_e4m3fn, torch.uint8), x.numel())
+    _require(scale, "scale", (torch.float32,), rows)
     _check(lib().dit_attn_quantize_e4m3_rows(x.data_ptr(), amax.data_ptr(), q.data_ptr(), scale.data_ptr(), rows,
                                              x.numel() // max(rows, 1), _stream_handle(stream)),
            "dit_attn_quantize_e4m3_rows")
@@ -416,15 +444,14 @@ def dit_attn_fwd_ulysses(q_shards, k_shards, v_shards, o_shards, lse_shards=None
         raise ValueError("one shard of each tensor per rank")
     B, H, Ls, D = q_shards[0].shape
     for t in (*q_shards, *k_shards, *v_shards):
-        if t.shape != (B, H, Ls, D) or t.dtype != q_shards[0].dtype or not t.is_contiguous():
-            raise ValueError("q/k/v shards must be contiguous [B, H, Ls, D] tensors of one dtype")
+        _require(t, "every q/k/v shard", (q_shards[0].dtype,))
+        if t.shape != (B, H, Ls, D):
+            raise ValueError("q/k/v shards must all be [B, H, Ls, D]")
     for t in o_shards:
-        if t.shape != (B, H, Ls, D) or t.dtype != torch.bfloat16 or not t.is_contiguous():
-            raise ValueError("o shards must be contiguous bf16 [B, H, Ls, D] tensors")
+        _require(t, "every o shard", (torch.bfloat16,), B * H * Ls * D)
     if lse_shards is not None:
         for t in lse_shards:
-            if t.numel() != B * H * Ls or t.dtype != torch.float32 or not t.is_contiguous():
-                raise ValueError("lse shards must be contiguous fp32 tensors of B*H*Ls elements")
+            _require(t, "every lse shard", (torch.float32,), B * H * Ls)
     if q_shards[0].dtype == torch.bfloat16:
         dtype, scales = DIT_ATTN_BF16, (None, None, None)
     elif q_shards[0].dtype == torch.float8_e4m3fn:

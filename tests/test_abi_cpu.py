@@ -179,3 +179,30 @@ def test_fused_ulysses_argument_validation(L):
     assert call(two, two, two, two, None, 0, 1, 4, 64, 96, 0.1, 0) == 2          # head dim
     assert call(two, two, two, two, None, 0, 1, 4, 64, 64, 0.1, 1) == 1          # FP8 without scales
     assert call(two, two, two, two, None, 0, 1, 4, 64, 64, -1.0, 0) == 8         # negative scale
+
+
+def test_python_bindings_refuse_host_buffers_before_any_call():
+    """Every caller-provided buffer must be a CUDA tensor: a host pointer reaching a kernel
+    would fault.  (On this host nothing is a CUDA tensor, so each check fires on the first
+    host tensor it meets.)"""
+    import attention_dit_attn_b200 as d
+    x = torch.zeros(64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        d.dit_attn_block_transpose(x, 2, 2)
+    with pytest.raises(ValueError):
+        d.dit_attn_absmax_rows(x, 4)
+    with pytest.raises(ValueError):
+        d.dit_attn_quantize_e4m3_rows(x, torch.ones(4))
+    with pytest.raises(ValueError):
+        d.dit_attn_residual_diff(x, x)
+    with pytest.raises(ValueError):
+        d.dit_attn_mxfp4_quantize(x.reshape(2, 32))
+    shard = torch.zeros((1, 2, 64, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        d.dit_attn_fwd_ulysses([shard], [shard], [shard], [shard.clone()], rank=0)
+
+
+def test_require_names_the_buffer_and_its_expected_form():
+    import attention_dit_attn_b200 as d
+    with pytest.raises(ValueError, match="diff must be a contiguous CUDA tensor of dtype torch.float32 with 1 elements"):
+        d._require(torch.zeros(1), "diff", (torch.float32,), 1)
