@@ -121,6 +121,9 @@ def ulysses_attention_fused(q, k, v, *, group=None, scale: float | None = None, 
     N = dist.get_world_size(group)
     rank = dist.get_rank(group)
     B, H, Ls, D = q.shape
+    # Checked before any collective, so every rank fails the same way.
+    if H % N or Ls % 64 or N > 8:
+        raise ValueError(f"need H % ranks == 0, Ls % 64 == 0 and at most 8 ranks (H={H}, Ls={Ls}, ranks={N})")
     o = torch.empty((B, H, Ls, D), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, H, Ls), dtype=torch.float32, device=q.device)
     local = [t.contiguous() for t in (q, k, v)] + [o, lse]
