@@ -76,3 +76,38 @@ def test_sharded_ulysses_equals_full_attention(world, fp8):
     o_ref, lse_ref = ops.attention(q, k, v, 1 / math.sqrt(D), *scales)
     assert torch.equal(o.view(torch.int16), o_ref.view(torch.int16))
     assert torch.equal(lse, lse_ref)
+
+
+def _fused_bad_shape_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+    from attention_dit_attn_b200.ulysses import ulysses_attention_fused
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=30))
+    try:
+        x = torch.zeros((1, 3, 64, 64), dtype=torch.bfloat16)          # 3 heads over 2 ranks
+        try:
+            ulysses_attention_fused(x, x, x)
+            out.put((rank, "returned"))
+        except ValueError:
+            out.put((rank, "ValueError"))
+        dist.barrier()                                                  # both ranks are still in step
+    finally:
+        dist.destroy_process_group()
+
+
+def test_fused_path_rejects_bad_shapes_on_every_rank_before_any_collective():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q_ = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_fused_bad_shape_main, args=(r, world, port, q_)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted(q_.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert got == [(0, "ValueError"), (1, "ValueError")]
