@@ -28,7 +28,8 @@ __all__ = [
     "dit_attn_residual_diff_ptr", "dit_attn_residual_diff_workspace_bytes", "dit_attn_residual_diff_noalloc",
     "dit_attn_mxfp4_quantize", "dit_attn_mxfp4_quantize_ptr", "dit_attn_block_transpose",
     "dit_attn_absmax_rows", "dit_attn_quantize_e4m3_rows", "dit_attn_fwd_ulysses", "dit_attn_fwd_ulysses_ptr",
-    "dit_attn_ulysses_check_device_error",
+    "dit_attn_ulysses_check_device_error", "dit_attn_gemm_fp8", "dit_attn_gemm_fp8_ptr",
+    "dit_attn_gemm_check_device_error",
     "ensure_built", "lib",
     "header_functions", "STATUS",
 ]
@@ -40,7 +41,7 @@ DIT_ATTN_MERGE_MAX_PARTS = 8
 STATUS = {
     0: "DIT_ATTN_OK", 1: "DIT_ATTN_ERR_NULL", 2: "DIT_ATTN_ERR_SHAPE", 3: "DIT_ATTN_ERR_DTYPE",
     4: "DIT_ATTN_ERR_ALIGN", 5: "DIT_ATTN_ERR_ARCH", 6: "DIT_ATTN_ERR_LAUNCH",
-    7: "DIT_ATTN_ERR_TIMEOUT", 8: "DIT_ATTN_ERR_VALUE",
+    7: "DIT_ATTN_ERR_TIMEOUT", 8: "DIT_ATTN_ERR_VALUE", 9: "DIT_ATTN_ERR_DEVICE",
 }
 
 HEADER = os.path.join(_build.INCLUDE, "dit_attn.h")
@@ -103,6 +104,10 @@ def lib() -> ctypes.CDLL:
                                                                                 vp]
         L.dit_attn_ulysses_check_device_error.restype = i32
         L.dit_attn_ulysses_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.dit_attn_gemm_fp8.restype = i32
+        L.dit_attn_gemm_fp8.argtypes = [vp, vp, vp, ctypes.c_longlong, i32, i32, ctypes.c_float, ctypes.c_float, vp]
+        L.dit_attn_gemm_check_device_error.restype = i32
+        L.dit_attn_gemm_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         _lib = L
     return _lib
 
@@ -118,11 +123,24 @@ def dit_attn_status_string(status: int) -> str:
     return lib().dit_attn_status_string(int(status)).decode()
 
 
-def _stream_handle(stream) -> int:
+def _stream_handle(stream, device=None) -> int:
     import torch
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _one_device(*tensors):
+    """The one CUDA device all given tensors (None entries skipped) live on.  Every
+    call runs with that device current and on its stream: the library launches on
+    the current device, and a kernel given another GPU's memory would read it
+    across the link or fault."""
+    import torch
+    devs = {t.device for t in tensors if isinstance(t, torch.Tensor)}
+    if len(devs) != 1 or next(iter(devs)).type != "cuda":
+        raise ValueError("all tensors of one call must be on the same CUDA device, got "
+                         + ", ".join(sorted(str(d) for d in devs)))
+    return next(iter(devs))
 
 
 def dit_attn_fwd_ptr(q: int, k: int, v: int, o: int, lse: int | None, B: int, H: int, L: int,
@@ -175,9 +193,11 @@ def dit_attn_fwd(q, k, v, o=None, lse=None, *, scale: float | None = None, q_sca
         raise ValueError("lse must be a contiguous fp32 CUDA tensor with B*H*L elements")
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    rc = dit_attn_fwd_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                          None if lse is None else lse.data_ptr(), B, H, L, D, float(scale), dtype,
-                          *scales, stream=_stream_handle(stream))
+    dev = _one_device(q, k, v, o, lse, q_scale, k_scale, v_scale)
+    with torch.cuda.device(dev):
+        rc = dit_attn_fwd_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              None if lse is None else lse.data_ptr(), B, H, L, D, float(scale), dtype,
+                              *scales, stream=_stream_handle(stream, dev))
     if rc != 0:
         raise DitAttnError(rc, "dit_attn_fwd: ")
     return o, lse
@@ -242,9 +262,11 @@ def dit_attn_lse_merge(parts, o=None, lse=None, *, want_lse: bool = True, stream
     elif lse is not None and (lse.numel() != rows or lse.dtype != torch.float32
                               or not lse.is_contiguous() or not lse.is_cuda):
         raise ValueError("lse must be a contiguous fp32 CUDA tensor with one value per row")
-    rc = dit_attn_lse_merge_ptr([oc.data_ptr() for oc, _ in parts], [lc.data_ptr() for _, lc in parts],
-                                o.data_ptr(), None if lse is None else lse.data_ptr(), rows, D,
-                                _stream_handle(stream))
+    dev = _one_device(o, lse, *[t for part in parts for t in part])
+    with torch.cuda.device(dev):
+        rc = dit_attn_lse_merge_ptr([oc.data_ptr() for oc, _ in parts], [lc.data_ptr() for _, lc in parts],
+                                    o.data_ptr(), None if lse is None else lse.data_ptr(), rows, D,
+                                    _stream_handle(stream, dev))
     if rc != 0:
         raise DitAttnError(rc, "dit_attn_lse_merge: ")
     return o, lse
@@ -288,8 +310,11 @@ def dit_attn_residual_diff(cur, prev, threshold: float = 0.12, *, workspace=None
         reuse = torch.empty(1, dtype=torch.int32, device=cur.device)
     _require(diff, "diff", (torch.float32,), 1)
     _require(reuse, "reuse", (torch.int32,), 1)
-    rc = dit_attn_residual_diff_ptr(cur.data_ptr(), prev.data_ptr(), n, float(threshold), workspace.data_ptr(),
-                                    workspace.numel(), diff.data_ptr(), reuse.data_ptr(), _stream_handle(stream))
+    dev = _one_device(cur, prev, workspace, diff, reuse)
+    with torch.cuda.device(dev):
+        rc = dit_attn_residual_diff_ptr(cur.data_ptr(), prev.data_ptr(), n, float(threshold),
+                                        workspace.data_ptr(), workspace.numel(), diff.data_ptr(), reuse.data_ptr(),
+                                        _stream_handle(stream, dev))
     if rc != 0:
         raise DitAttnError(rc, "dit_attn_residual_diff: ")
     return diff, reuse
@@ -311,8 +336,11 @@ def dit_attn_residual_diff_noalloc(cur, prev, threshold: float = 0.12, *, diff=N
         reuse = torch.empty(1, dtype=torch.int32, device=cur.device)
     _require(diff, "diff", (torch.float32,), 1)
     _require(reuse, "reuse", (torch.int32,), 1)
-    rc = lib().dit_attn_residual_diff_noalloc(cur.data_ptr(), prev.data_ptr(), cur.numel(), ctypes.c_float(threshold),
-                                              diff.data_ptr(), reuse.data_ptr(), _stream_handle(stream))
+    dev = _one_device(cur, prev, diff, reuse)
+    with torch.cuda.device(dev):
+        rc = lib().dit_attn_residual_diff_noalloc(cur.data_ptr(), prev.data_ptr(), cur.numel(),
+                                                  ctypes.c_float(threshold), diff.data_ptr(), reuse.data_ptr(),
+                                                  _stream_handle(stream, dev))
     if rc != 0:
         raise DitAttnError(rc, "dit_attn_residual_diff_noalloc: ")
     return diff, reuse
@@ -339,7 +367,10 @@ def dit_attn_mxfp4_quantize(x, q=None, scales=None, *, stream=None):
     for name, t, cols in (("q", q, K // 2), ("scales", scales, K // 32)):
         if not (t.is_cuda and t.dtype == torch.uint8 and t.is_contiguous() and t.numel() == rows * cols):
             raise ValueError(f"{name} must be a contiguous uint8 CUDA tensor with {rows * cols} elements")
-    rc = dit_attn_mxfp4_quantize_ptr(x.data_ptr(), q.data_ptr(), scales.data_ptr(), rows, K, _stream_handle(stream))
+    dev = _one_device(x, q, scales)
+    with torch.cuda.device(dev):
+        rc = dit_attn_mxfp4_quantize_ptr(x.data_ptr(), q.data_ptr(), scales.data_ptr(), rows, K,
+                                         _stream_handle(stream, dev))
     if rc != 0:
         raise DitAttnError(rc, "dit_attn_mxfp4_quantize: ")
     return q, scales
@@ -377,8 +408,10 @@ def dit_attn_block_transpose(x, R: int, C: int, out=None, *, stream=None):
     if out is None:
         out = torch.empty_like(x)
     _require(out, "out", nbytes=nbytes)
-    _check(lib().dit_attn_block_transpose(x.data_ptr(), out.data_ptr(), R, C, nbytes // (R * C),
-                                          _stream_handle(stream)), "dit_attn_block_transpose")
+    dev = _one_device(x, out)
+    with torch.cuda.device(dev):
+        _check(lib().dit_attn_block_transpose(x.data_ptr(), out.data_ptr(), R, C, nbytes // (R * C),
+                                              _stream_handle(stream, dev)), "dit_attn_block_transpose")
     return out
 
 
@@ -392,8 +425,10 @@ def dit_attn_absmax_rows(x, rows: int, out=None, *, stream=None):
     if out is None:
         out = torch.empty(rows, dtype=torch.float32, device=x.device)
     _require(out, "out", (torch.float32,), rows)
-    _check(lib().dit_attn_absmax_rows(x.data_ptr(), out.data_ptr(), rows, x.numel() // max(rows, 1),
-                                      _stream_handle(stream)), "dit_attn_absmax_rows")
+    dev = _one_device(x, out)
+    with torch.cuda.device(dev):
+        _check(lib().dit_attn_absmax_rows(x.data_ptr(), out.data_ptr(), rows, x.numel() // max(rows, 1),
+                                          _stream_handle(stream, dev)), "dit_attn_absmax_rows")
     return out
 
 
@@ -413,9 +448,11 @@ def dit_attn_quantize_e4m3_rows(x, amax, q=None, scale=None, *, stream=None):
         scale = torch.empty(rows, dtype=torch.float32, device=x.device)
     _require(q, "q", (torch.float8_e4m3fn, torch.uint8), x.numel())
     _require(scale, "scale", (torch.float32,), rows)
-    _check(lib().dit_attn_quantize_e4m3_rows(x.data_ptr(), amax.data_ptr(), q.data_ptr(), scale.data_ptr(), rows,
-                                             x.numel() // max(rows, 1), _stream_handle(stream)),
-           "dit_attn_quantize_e4m3_rows")
+    dev = _one_device(x, amax, q, scale)
+    with torch.cuda.device(dev):
+        _check(lib().dit_attn_quantize_e4m3_rows(x.data_ptr(), amax.data_ptr(), q.data_ptr(), scale.data_ptr(),
+                                                 rows, x.numel() // max(rows, 1), _stream_handle(stream, dev)),
+               "dit_attn_quantize_e4m3_rows")
     return q, scale
 
 
@@ -465,10 +502,17 @@ def dit_attn_fwd_ulysses(q_shards, k_shards, v_shards, o_shards, lse_shards=None
         raise TypeError(f"unsupported dtype {q_shards[0].dtype}")
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    if not 0 <= rank < n:
+        raise ValueError(f"rank {rank} outside 0..{n - 1}")
+    # Peers' shards may live on other GPUs (mapped into this context); the call
+    # runs on the device of this rank's own shards, where the scales live too.
+    own = [q_shards[rank], k_shards[rank], v_shards[rank], o_shards[rank]]
+    dev = _one_device(*own, None if lse_shards is None else lse_shards[rank], q_scale, k_scale, v_scale)
     ptrs = lambda ts: [t.data_ptr() for t in ts]
-    rc = dit_attn_fwd_ulysses_ptr(ptrs(q_shards), ptrs(k_shards), ptrs(v_shards), ptrs(o_shards),
-                                  None if lse_shards is None else ptrs(lse_shards), rank, B, H, Ls, D, float(scale),
-                                  dtype, *scales, stream=_stream_handle(stream))
+    with torch.cuda.device(dev):
+        rc = dit_attn_fwd_ulysses_ptr(ptrs(q_shards), ptrs(k_shards), ptrs(v_shards), ptrs(o_shards),
+                                      None if lse_shards is None else ptrs(lse_shards), rank, B, H, Ls, D,
+                                      float(scale), dtype, *scales, stream=_stream_handle(stream, dev))
     _check(rc, "dit_attn_fwd_ulysses")
 
 
@@ -476,4 +520,38 @@ def dit_attn_ulysses_check_device_error(stream=None) -> tuple[int, int]:
     """The fused Ulysses kernel's device error word: synchronise, read, clear: (status, raw word)."""
     word = ctypes.c_uint32(0)
     rc = lib().dit_attn_ulysses_check_device_error(_stream_handle(stream), ctypes.byref(word))
+    return rc, word.value
+
+
+def dit_attn_gemm_fp8_ptr(a: int, w: int, y: int, M: int, N: int, K: int, a_scale: float, w_scale: float,
+                          stream: int = 0) -> int:
+    """Raw C-ABI call with integer device pointers; returns the status code."""
+    return lib().dit_attn_gemm_fp8(a, w, y, M, N, K, ctypes.c_float(a_scale), ctypes.c_float(w_scale), stream)
+
+
+def dit_attn_gemm_fp8(a, w, a_scale: float, w_scale: float, y=None, *, stream=None):
+    """FP8 linear layer y = a_scale * w_scale * (a @ w^T): a [..., K] and w [N, K] float8_e4m3fn
+    (or uint8 codes) CUDA tensors, y bf16 [..., N] (allocated when not given).
+    Asynchronous on ``stream``."""
+    import torch
+    for name, t in (("a", a), ("w", w)):
+        _require(t, name, (torch.float8_e4m3fn, torch.uint8))
+    if w.dim() != 2 or a.shape[-1] != w.shape[1]:
+        raise ValueError("w must be [N, K] with K = a.shape[-1]")
+    N, K = w.shape
+    M = a.numel() // K if K else 0
+    if y is None:
+        y = torch.empty(tuple(a.shape[:-1]) + (N,), dtype=torch.bfloat16, device=a.device)
+    _require(y, "y", (torch.bfloat16,), M * N)
+    dev = _one_device(a, w, y)
+    with torch.cuda.device(dev):
+        _check(dit_attn_gemm_fp8_ptr(a.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, float(a_scale),
+                                     float(w_scale), _stream_handle(stream, dev)), "dit_attn_gemm_fp8")
+    return y
+
+
+def dit_attn_gemm_check_device_error(stream=None) -> tuple[int, int]:
+    """The GEMM kernels' device error word: synchronise, read, clear: (status, raw word)."""
+    word = ctypes.c_uint32(0)
+    rc = lib().dit_attn_gemm_check_device_error(_stream_handle(stream), ctypes.byref(word))
     return rc, word.value

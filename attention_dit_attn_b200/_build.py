@@ -10,9 +10,11 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdit_attn.so")
-SOURCES = ["dit_attn.cu", "lse_merge.cu", "residual_diff.cu", "mxfp4_quant.cu", "ulysses_ops.cu", "ulysses_fused.cu"]
+SOURCES = ["dit_attn.cu", "lse_merge.cu", "residual_diff.cu", "mxfp4_quant.cu", "ulysses_ops.cu", "ulysses_fused.cu",
+           "lowp_gemm.cu"]
 DEPS = ["dit_attn.cu", "lse_merge.cu", "residual_diff.cu", "mxfp4_quant.cu", "ulysses_ops.cu", "ulysses_fused.cu",
-        "attn_common.cuh", "attn_fwd_sm100.cuh", "attn_fwd_ulysses_sm100.cuh", "sm100_ptx.cuh"]
+        "attn_common.cuh", "attn_fwd_sm100.cuh", "attn_fwd_ulysses_sm100.cuh", "sm100_ptx.cuh", "abi_util.h",
+        "lowp_gemm.cu", "gemm_sm100.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

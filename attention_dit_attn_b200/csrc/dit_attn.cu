@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "abi_util.h"
 #include "dit_attn.h"
 #include "attn_fwd_sm100.cuh"
 
@@ -57,6 +58,32 @@ CUtensorMapSwizzle swizzle_for(int bytes)
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_attr_set[4][kMaxDevices];
 
+// The four tensor maps of a call depend only on (device, q, k, v, o, B*H, L,
+// variant): a small cache lets a repeated call (every layer and denoising step
+// of a DiT) skip the four cuTensorMapEncodeTiled calls.  A map holds nothing
+// but the address, shape and strides, so an entry stays valid for any buffer
+// at the same address with the same shape.
+struct MapKey {
+    int device, variant, L;
+    long long BH;
+    const void *q, *k, *v, *o;
+    bool operator==(const MapKey &b) const
+    {
+        return device == b.device && variant == b.variant && L == b.L && BH == b.BH && q == b.q && k == b.k &&
+               v == b.v && o == b.o;
+    }
+};
+struct MapEntry {
+    MapKey key;
+    CUtensorMap tq, tk, tv, to;
+    unsigned long long used;
+    bool valid;
+};
+constexpr int kMapCache = 16;
+std::mutex g_map_mu;
+MapEntry g_maps[kMapCache];
+unsigned long long g_map_clock = 0;
+
 // Clusters of 2 CTAs, one 128-row query tile per CTA.
 template <int D, bool FP8>
 int launch(const void *q, const void *k, const void *v, void *o, const dit::FwdParams &prm,
@@ -72,14 +99,37 @@ int launch(const void *q, const void *k, const void *v, void *o, const dit::FwdP
         if (device < kMaxDevices)
             g_attr_set[variant][device].store(1, std::memory_order_release);
     }
-    const CUtensorMapDataType in_t = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const MapKey key{device, variant, L, BH, q, k, v, o};
     CUtensorMap tq, tk, tv, to;
-    if (!make_map(&tq, q, in_t, C::ELT, D, L, BH, C::BOX_ELEMS, swizzle_for(C::SWZ), dit::kBM) ||
-        !make_map(&tk, k, in_t, C::ELT, D, L, BH, C::BOX_ELEMS, swizzle_for(C::SWZ), C::KROWS) ||
-        !make_map(&tv, v, in_t, C::ELT, D, L, BH, D / 2, swizzle_for(C::VRAW_ROW), dit::kBN) ||
-        !make_map(&to, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, L, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B,
-                  dit::kBM))
-        return DIT_ATTN_ERR_LAUNCH;
+    bool hit = false;
+    {
+        std::lock_guard<std::mutex> lock(g_map_mu);
+        for (MapEntry &e : g_maps)
+            if (e.valid && e.key == key) {
+                tq = e.tq, tk = e.tk, tv = e.tv, to = e.to;
+                e.used = ++g_map_clock;
+                hit = true;
+                break;
+            }
+    }
+    if (!hit) {
+        const CUtensorMapDataType in_t = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        if (!make_map(&tq, q, in_t, C::ELT, D, L, BH, C::BOX_ELEMS, swizzle_for(C::SWZ), dit::kBM) ||
+            !make_map(&tk, k, in_t, C::ELT, D, L, BH, C::BOX_ELEMS, swizzle_for(C::SWZ), C::KROWS) ||
+            !make_map(&tv, v, in_t, C::ELT, D, L, BH, D / 2, swizzle_for(C::VRAW_ROW), dit::kBN) ||
+            !make_map(&to, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, L, BH, 64, CU_TENSOR_MAP_SWIZZLE_128B,
+                      dit::kBM))
+            return DIT_ATTN_ERR_LAUNCH;
+        std::lock_guard<std::mutex> lock(g_map_mu);
+        MapEntry *slot = &g_maps[0];
+        for (MapEntry &e : g_maps)
+            if (!e.valid || e.used < slot->used) {
+                slot = &e;
+                if (!e.valid)
+                    break;
+            }
+        *slot = MapEntry{key, tq, tk, tv, to, ++g_map_clock, true};
+    }
     const long long blocks = 2 * BH * (long long)prm.n_pairs;
     if (blocks > 0x7FFFFFFFll)
         return DIT_ATTN_ERR_SHAPE;
@@ -145,6 +195,8 @@ int dit_attn_fwd(const void *q, const void *k, const void *v, void *o, float *ls
     const int dev_rc = check_device(&device);
     if (dev_rc != DIT_ATTN_OK)
         return dev_rc;
+    if (!dit_abi::device_buffers(device, {q, k, v, o, lse, q_scale, k_scale, v_scale}))
+        return DIT_ATTN_ERR_DEVICE;
 
     dit::FwdParams prm{};
     prm.L = L;
@@ -179,6 +231,8 @@ const char *dit_attn_status_string(int status)
     case DIT_ATTN_ERR_LAUNCH: return "a CUDA runtime call or the kernel launch failed";
     case DIT_ATTN_ERR_TIMEOUT: return "a device-side wait exceeded its time limit";
     case DIT_ATTN_ERR_VALUE: return "scale must be finite and >= 0";
+    case DIT_ATTN_ERR_DEVICE:
+        return "a buffer is not device memory of the current device (host memory, another GPU's, or unallocated)";
     default: return "unknown status";
     }
 }

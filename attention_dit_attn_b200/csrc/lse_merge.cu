@@ -21,6 +21,7 @@
 #include <cmath>
 #include <cstdint>
 
+#include "abi_util.h"
 #include "dit_attn.h"
 
 namespace {
@@ -179,7 +180,9 @@ cudaError_t launch_n(const MergeParams &p, int vpr, int sms, cudaStream_t stream
     return vpr == 16 ? launch_nv<N, 16>(p, sms, stream) : launch_nv<N, 8>(p, sms, stream);
 }
 
-std::atomic<int> g_sm_count{0};
+// SM count per device, looked up once per device.
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -214,11 +217,18 @@ extern "C" int dit_attn_lse_merge(const void *const *o_parts, const float *const
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess ||
         major != 10 || minor != 0)
         return DIT_ATTN_ERR_ARCH;
-    int sms = g_sm_count.load(std::memory_order_relaxed);
+    if (device >= kMaxDevices)
+        return DIT_ATTN_ERR_ARCH;
+    if (!dit_abi::device_buffers(device, {o, lse}))
+        return DIT_ATTN_ERR_DEVICE;
+    for (int c = 0; c < n_parts; ++c)
+        if (!dit_abi::device_buffers(device, {o_parts[c], lse_parts[c]}))
+            return DIT_ATTN_ERR_DEVICE;
+    int sms = g_sm_count[device].load(std::memory_order_relaxed);
     if (sms == 0) {
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
             return DIT_ATTN_ERR_LAUNCH;
-        g_sm_count.store(sms, std::memory_order_relaxed);
+        g_sm_count[device].store(sms, std::memory_order_relaxed);
     }
     MergeParams p{};
     for (int c = 0; c < n_parts; ++c) {

@@ -21,6 +21,7 @@
 #include <atomic>
 #include <cstdint>
 
+#include "abi_util.h"
 #include "dit_attn.h"
 
 namespace {
@@ -111,7 +112,9 @@ __global__ void __launch_bounds__(kThreads) mxfp4_quant_kernel(const QuantParams
     }
 }
 
-std::atomic<int> g_resident{0};
+// Resident blocks per device (occupancy x SM count), looked up once per device.
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_resident[kMaxDevices];
 
 bool aligned(const void *q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) == 0; }
 
@@ -134,7 +137,11 @@ extern "C" int dit_attn_mxfp4_quantize(const void *x, void *q, void *scales, lon
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess ||
         major != 10 || minor != 0)
         return DIT_ATTN_ERR_ARCH;
-    int resident = g_resident.load(std::memory_order_relaxed);
+    if (device >= kMaxDevices)
+        return DIT_ATTN_ERR_ARCH;
+    if (!dit_abi::device_buffers(device, {x, q, scales}))
+        return DIT_ATTN_ERR_DEVICE;
+    int resident = g_resident[device].load(std::memory_order_relaxed);
     if (resident == 0) {
         int sms = 0, per_sm = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
@@ -142,7 +149,7 @@ extern "C" int dit_attn_mxfp4_quantize(const void *x, void *q, void *scales, lon
                 cudaSuccess)
             return DIT_ATTN_ERR_LAUNCH;
         resident = (per_sm > 0 ? per_sm : 1) * sms;
-        g_resident.store(resident, std::memory_order_relaxed);
+        g_resident[device].store(resident, std::memory_order_relaxed);
     }
     QuantParams p{};
     p.x = static_cast<const uint4 *>(x);

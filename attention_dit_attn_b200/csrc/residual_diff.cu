@@ -15,12 +15,15 @@
 // ticket) adds the partials in a fixed order in fp64, takes the decision,
 // writes diff and the flag, and resets the ticket, so the result is
 // bit-reproducible and the workspace is left ready for the next call.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
+#include "abi_util.h"
 #include "dit_attn.h"
 
 namespace {
@@ -153,16 +156,55 @@ int blocks_for(long long n, int resident)
     return (int)(want < 1 ? 1 : (want < cap ? want : cap));
 }
 
-std::atomic<int> g_resident{0};
+// Resident blocks per device (occupancy x SM count), looked up once per device.
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_resident[kMaxDevices];
 
 // Scratch of the no-allocation entry point: the largest workspace any n needs,
 // in the module's own device memory (zero at load; every call leaves it zero).
 constexpr size_t kScratchBytes = kHeaderBytes + sizeof(double2) * kMaxBlocks;
 static __device__ __align__(256) unsigned char g_diff_scratch[kScratchBytes];
 
-// Its address per device, looked up once.
-constexpr int kMaxDevices = 64;
-std::atomic<void *> g_scratch_addr[kMaxDevices];
+// Its address per device, looked up once per CUDA context: a context made
+// after cudaDeviceReset loads the module again, at a new address.  Contexts
+// are told apart by their process-unique id (cuCtxGetId), never reused.
+struct ScratchAddr {
+    unsigned long long ctx_id;
+    void *addr;
+};
+std::mutex g_scratch_mu;
+ScratchAddr g_scratch_addr[kMaxDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+template <class Fn>
+Fn driver_fn(const char *name)
+{
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) == cudaSuccess && q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<Fn>(ptr);
+    return nullptr;
+}
+
+// Id of the context current on this thread (0 when none can be had).
+unsigned long long current_ctx_id()
+{
+    static std::once_flag once;
+    static CtxGetCurrentFn get_ctx = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    std::call_once(once, [] {
+        get_ctx = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+        get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    // cudaFree(0) makes the device's primary context current if none is yet.
+    if (get_ctx == nullptr || get_id == nullptr || cudaFree(0) != cudaSuccess || get_ctx(&ctx) != CUDA_SUCCESS ||
+        ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id + 1;   // 0 stays "none"
+}
 
 bool aligned(const void *q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) == 0; }
 
@@ -196,7 +238,11 @@ extern "C" int dit_attn_residual_diff(const void *cur, const void *prev, long lo
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess ||
         major != 10 || minor != 0)
         return DIT_ATTN_ERR_ARCH;
-    int resident = g_resident.load(std::memory_order_relaxed);
+    if (device >= kMaxDevices)
+        return DIT_ATTN_ERR_ARCH;
+    if (!dit_abi::device_buffers(device, {cur, prev, workspace, diff_out, reuse_out}))
+        return DIT_ATTN_ERR_DEVICE;
+    int resident = g_resident[device].load(std::memory_order_relaxed);
     if (resident == 0) {
         int sms = 0, per_sm = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
@@ -204,7 +250,7 @@ extern "C" int dit_attn_residual_diff(const void *cur, const void *prev, long lo
                 cudaSuccess)
             return DIT_ATTN_ERR_LAUNCH;
         resident = (per_sm > 0 ? per_sm : 1) * sms;
-        g_resident.store(resident, std::memory_order_relaxed);
+        g_resident[device].store(resident, std::memory_order_relaxed);
     }
     DiffParams p{};
     p.cur = static_cast<const uint4 *>(cur);
@@ -227,11 +273,22 @@ extern "C" int dit_attn_residual_diff_noalloc(const void *cur, const void *prev,
     int device = 0;
     if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices)
         return DIT_ATTN_ERR_ARCH;
-    void *scratch = g_scratch_addr[device].load(std::memory_order_acquire);
-    if (scratch == nullptr) {
-        if (cudaGetSymbolAddress(&scratch, g_diff_scratch) != cudaSuccess)
-            return DIT_ATTN_ERR_ARCH;
-        g_scratch_addr[device].store(scratch, std::memory_order_release);
+    const unsigned long long ctx_id = current_ctx_id();
+    if (ctx_id == 0)
+        return DIT_ATTN_ERR_ARCH;
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_scratch_mu);
+        ScratchAddr &slot = g_scratch_addr[device];
+        if (slot.ctx_id != ctx_id || slot.addr == nullptr) {
+            if (cudaGetSymbolAddress(&slot.addr, g_diff_scratch) != cudaSuccess) {
+                slot.addr = nullptr;
+                slot.ctx_id = 0;
+                return DIT_ATTN_ERR_ARCH;
+            }
+            slot.ctx_id = ctx_id;
+        }
+        scratch = slot.addr;
     }
     return dit_attn_residual_diff(cur, prev, n, threshold, scratch, kScratchBytes, diff_out, reuse_out, stream);
 }

@@ -19,6 +19,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "abi_util.h"
 #include "dit_attn.h"
 #include "attn_fwd_ulysses_sm100.cuh"
 
@@ -161,6 +162,15 @@ int dit_attn_fwd_ulysses(const void *const *q_shards, const void *const *k_shard
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess ||
         major != 10 || minor != 0)
         return DIT_ATTN_ERR_ARCH;
+    // Shards may be peers' memory mapped into this context; the scales are
+    // read by this device only.
+    for (int c = 0; c < n_ranks; ++c)
+        if (!dit_abi::device_buffers(device, {q_shards[c], k_shards[c], v_shards[c], o_shards[c],
+                                              with_lse ? lse_shards[c] : nullptr},
+                                     /*peers_ok=*/true))
+            return DIT_ATTN_ERR_DEVICE;
+    if (!dit_abi::device_buffers(device, {q_scale, k_scale, v_scale}))
+        return DIT_ATTN_ERR_DEVICE;
 
     dit::FwdParams prm{};
     prm.L = (int)L;

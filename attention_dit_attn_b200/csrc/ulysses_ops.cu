@@ -25,6 +25,7 @@
 #include <atomic>
 #include <cstdint>
 
+#include "abi_util.h"
 #include "dit_attn.h"
 
 namespace {
@@ -156,7 +157,8 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const uint4 *x,
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-int check_arch()
+// The current device is a B200 and every buffer is its device memory.
+int check_arch(std::initializer_list<const void *> buffers)
 {
     int device = 0, major = 0, minor = 0;
     if (cudaGetDevice(&device) != cudaSuccess ||
@@ -164,7 +166,7 @@ int check_arch()
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess ||
         major != 10 || minor != 0)
         return DIT_ATTN_ERR_ARCH;
-    return DIT_ATTN_OK;
+    return dit_abi::device_buffers(device, buffers) ? DIT_ATTN_OK : DIT_ATTN_ERR_DEVICE;
 }
 
 // Grid of a row-chunked kernel: chunks of `per_cta` units per row in x, rows
@@ -189,7 +191,7 @@ extern "C" int dit_attn_block_transpose(const void *in, void *out, long long R, 
         return DIT_ATTN_ERR_NULL;
     if (!aligned(in, 4) || !aligned(out, 4))
         return DIT_ATTN_ERR_ALIGN;
-    const int rc = check_arch();
+    const int rc = check_arch({in, out});
     if (rc != DIT_ATTN_OK)
         return rc;
     const bool wide = block_bytes % 16 == 0 && aligned(in, 16) && aligned(out, 16);
@@ -217,7 +219,7 @@ extern "C" int dit_attn_absmax_rows(const void *x, float *amax, long long rows, 
         return DIT_ATTN_ERR_NULL;
     if (!aligned(x, 16) || !aligned(amax, 4))
         return DIT_ATTN_ERR_ALIGN;
-    const int rc = check_arch();
+    const int rc = check_arch({x, amax});
     if (rc != DIT_ATTN_OK)
         return rc;
     if (cudaMemsetAsync(amax, 0, (size_t)rows * sizeof(float), stream) != cudaSuccess)
@@ -238,7 +240,7 @@ extern "C" int dit_attn_quantize_e4m3_rows(const void *x, const float *amax, voi
         return DIT_ATTN_ERR_NULL;
     if (!aligned(x, 16) || !aligned(q, 16) || !aligned(amax, 4) || (scale_out != nullptr && !aligned(scale_out, 4)))
         return DIT_ATTN_ERR_ALIGN;
-    const int rc = check_arch();
+    const int rc = check_arch({x, amax, q, scale_out});
     if (rc != DIT_ATTN_OK)
         return rc;
     quantize_rows_kernel<<<grid_rows(rows, row_len / 16, kUnitsPerCta), kThreads, 0, stream>>>(

@@ -157,3 +157,28 @@ def as_bits(t: torch.Tensor) -> np.ndarray:
     if t.dtype == torch.float8_e4m3fn:
         return t.contiguous().view(torch.uint8).numpy()
     raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# Linear-layer operands of the low-precision GEMMs: the DiT's QKV / output
+# projection shapes, M = B * L tokens by K = N = H * D features (FLUX: 3072).
+GEMM_SHAPES = {
+    "flux_2048_cfg_proj": (2 * (512 + 16384), 3072, 3072),     # (M, N, K)
+    "flux_1024x768_proj": (512 + 3072, 3072, 3072),
+}
+
+
+def gemm_operands_e4m3(M: int, N: int, K: int, seed: int = 0):
+    """A [M, K] and W [N, K] drawn N(0,1) (W scaled by 1/sqrt(K), as a trained
+    linear layer's weights are), each quantised per tensor to e4m3:
+    s = max|x| / 448, codes = e4m3(x / s) (nearest-even, torch's cast).
+    Returns (a codes, a_scale, w codes, w_scale); codes as torch.float8_e4m3fn."""
+    g = torch.Generator().manual_seed(int(seed))
+    a = torch.randn((M, K), generator=g, dtype=torch.float32)
+    w = torch.randn((N, K), generator=g, dtype=torch.float32) / math.sqrt(K)
+    out = []
+    for x in (a, w):
+        amax = float(x.abs().max())
+        s = amax / E4M3_MAX if amax > 0 else 1.0
+        s = float(torch.tensor(s, dtype=torch.float32))
+        out += [(x / s).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn), s]
+    return tuple(out)

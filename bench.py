@@ -12,8 +12,12 @@ hot path is one kernel launch).  Prints ONE JSON line on rank 0.
   from pinned host memory and o/lse copied back, inside the timed region.
 * roofline: the attention kernel against the measured bf16 (or derived fp8)
   tensor peak.
+* per_workload (N=1): the other configurations (flux_1024x768, sd35_1024_fp8,
+  wan_720p_81f), each device-timed for about a second with its own clock
+  record, TFLOP/s, % of nominal peak and roofline fraction.
 * cpu_baseline: the fp64 oracle on this host's cores over a bounded sample of
-  the workload's query rows (rank 0, N=1 only).
+  the workload's query rows, plus a one-thread run, the host's CPU model and
+  the extrapolated time of a full call (rank 0, N=1 only).
 * --impl reference: the oracle alone, as the reference arm, on the same
   workload and metric.
 * --op lse_merge: instead of the forward, the LSE merge of --parts partial
@@ -26,6 +30,9 @@ hot path is one kernel launch).  Prints ONE JSON line on rank 0.
   the previous step's); GB/s of algorithmic HBM traffic.
 * --op mxfp4_quant: the MXFP4 1x32 activation quantiser on a (B*L) x (H*D)
   bf16 activation of the workload; GB/s of algorithmic HBM traffic.
+* --op gemm_fp8: the FP8 linear layer Y = A W^T of the workload's projection
+  (M = B*L tokens, N = K = H*D features), e4m3 in, bf16 out; TFLOP/s,
+  roofline against the fp8 dense peak (2 x the measured bf16 peak).
 * --op ulysses_fp8_payload: the per-GPU preparation of Ulysses' FP8 all-to-all
   payload for one [B, H, L, D] bf16 tensor of the workload: per-head absmax,
   e4m3 quantisation, heads grouped by destination rank; GB/s of algorithmic
@@ -53,6 +60,7 @@ METRIC = "attention TFLOP/s and % of B200 tensor-core peak at 1 GPU"
 MERGE_METRIC = "LSE merge of partial attentions: GB/s of algorithmic HBM traffic at 1 GPU"
 DIFF_METRIC = "step-cache residual-change decision: GB/s of algorithmic HBM traffic at 1 GPU"
 MXFP4_METRIC = "MXFP4 1x32 activation quantiser: GB/s of algorithmic HBM traffic at 1 GPU"
+GEMM_FP8_METRIC = "FP8 linear layer Y = A W^T (e4m3 in, bf16 out): TFLOP/s at 1 GPU"
 PAYLOAD_METRIC = ("Ulysses FP8 payload preparation (absmax, e4m3 quantise, head grouping): "
                   "GB/s of algorithmic HBM traffic at 1 GPU")
 DEFAULT_WORKLOAD = "flux_2048_cfg"      # the first workload with L >= 16k (the stated target)
@@ -80,6 +88,7 @@ KERNEL_SOURCES = {
     "residual_diff": ["residual_diff.cu"],
     "mxfp4_quant": ["mxfp4_quant.cu"],
     "ulysses_ops": ["ulysses_ops.cu"],
+    "lowp_gemm": ["gemm_sm100.cuh", "lowp_gemm.cu", "sm100_ptx.cuh"],
 }
 
 
@@ -251,14 +260,37 @@ def plan_sample(w, inp, seconds: float):
     return w.L, heads
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(w, inp, seconds: float = 15.0):
+    """The oracle on all host threads (about `seconds`), then on one thread (about a
+    fifth of that), each on sampled query rows; the full call's time on this host is
+    extrapolated from the all-threads rate (4*L*D FLOPs per row, B*H*L rows)."""
     import oracle
     rows, heads = plan_sample(w, inp, seconds)
     dt, flops = oracle_sample_time(w, inp, rows, heads)
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+    rate = flops / dt
+    rows1 = max(16, min(w.L, int(rows * heads * 0.2 / oracle.max_threads()) or 16))
+    dt1, flops1 = oracle_sample_time(w, inp, rows1, 1, nthreads=1)
+    return {"value": rate / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
             "kind": "oracle",
             "sample": f"fp64 oracle on {rows} sampled query rows x {heads} head(s) of batch 0 of "
-                      f"{w.name} (all {w.L} keys per row): {dt:.1f} s on {oracle.max_threads()} threads"}
+                      f"{w.name} (all {w.L} keys per row): {dt:.1f} s on {oracle.max_threads()} threads",
+            "single_thread": {"value": flops1 / dt1 / 1e12, "unit": "TFLOP/s",
+                              "sample": f"{rows1} sampled query rows of head 0: {dt1:.2f} s on 1 thread"},
+            "host_cpus": os.cpu_count(), "cpu_model": cpu_model(),
+            "full_call_seconds_extrapolated": w.flops / rate,
+            "full_call_note": f"all {w.B * w.H * w.L} query rows of one call at the sampled all-threads rate"}
 
 
 # ------------------------------------------------------------------ arms
@@ -809,6 +841,167 @@ def run_mxfp4(args, dist: Dist):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ FP8 linear-layer GEMM (NEXT-3)
+
+def gemm_shape(w):
+    """The DiT block's projection on this workload: M = B*L tokens, N = K = H*D features."""
+    return w.B * w.L, w.H * w.D, w.H * w.D
+
+
+def gemm_config(w, M, N, K):
+    in_bytes = M * K + N * K
+    return {"workload": w.name, "op": "gemm_fp8", "M": M, "N": N, "K": K, "input_dtype": "e4m3",
+            "output_dtype": "bf16", "flops_per_call": 2.0 * M * N * K,
+            "bytes_per_call": in_bytes + 2 * M * N,
+            "l2": "inputs and output larger than L2" if in_bytes + 2 * M * N > L2_BYTES
+            else "L2 flushed between timed steps (256 MB write)",
+            "parallelism": "replicas"}
+
+
+def gemm_oracle_rate(a, sa, w_, sw, seconds: float):
+    """fp64 oracle (oracle/lowp_gemm.py) on the first rows of A: (TFLOP/s, rows, s)."""
+    import torch
+    from oracle import lowp_gemm
+    ac, wc = a.view(torch.uint8).numpy(), w_.view(torch.uint8).numpy()
+    rows = 4
+    while True:
+        t0 = time.perf_counter()
+        lowp_gemm.gemm_e4m3(ac[:rows], sa, wc, sw)
+        dt = time.perf_counter() - t0
+        if dt >= seconds / 4 or rows >= ac.shape[0]:
+            return 2.0 * rows * wc.shape[0] * wc.shape[1] / dt / 1e12, rows, dt
+        rows = min(ac.shape[0], rows * 4)
+
+
+def run_gemm_reference(args, dist: Dist):
+    if dist.rank != 0:
+        return
+    from attention_dit_attn_b200 import workloads as wl
+    w = wl.ALL[args.workload]
+    M, N, K = gemm_shape(w)
+    a, sa, w_, sw = wl.gemm_operands_e4m3(min(M, 1024), N, K, seed=w.seed)
+    per = 60.0 / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        gemm_oracle_rate(a, sa, w_, sw, per)
+    rates = [gemm_oracle_rate(a, sa, w_, sw, per) for _ in range(args.steps)]
+    value = statistics.median(r[0] for r in rates)
+    line = {
+        "impl": "reference", "metric": GEMM_FP8_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * 2.0 * M * N * K / (value * 1e12),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": gemm_config(w, M, N, K),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"each step: fp64 numpy oracle (BLAS) on {rates[0][1]} rows of A x [{N}, {K}]"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_gemm(args, dist: Dist):
+    import torch
+    import attention_dit_attn_b200 as dit
+    from attention_dit_attn_b200 import workloads as wl
+
+    dit.ensure_built()
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    w = wl.ALL[args.workload]
+    M, N, K = gemm_shape(w)
+    a_cpu, sa, w_cpu, sw = wl.gemm_operands_e4m3(M, N, K, seed=w.seed)
+    a, wt = a_cpu.to(dev), w_cpu.to(dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    cfg = gemm_config(w, M, N, K)
+    flops = cfg["flops_per_call"]
+    flush = None
+    if cfg["bytes_per_call"] <= L2_BYTES:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda aa, yy: dit.dit_attn_gemm_fp8(aa, wt, sa, sw, y=yy, stream=stream)
+    for _ in range(args.warmup):
+        call(a, y)
+    torch.cuda.synchronize(dev)
+    rc, word = dit.dit_attn_gemm_check_device_error(stream)
+    if rc != 0:
+        raise RuntimeError(f"device error during warm-up: {word:#x}")
+    sampler = ClockSampler()
+    if dist.rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for e0, e1 in evs:
+        if flush is not None:
+            flush.fill_(1)
+        e0.record(stream)
+        call(a, y)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    seconds = sum(e0.elapsed_time(e1) for e0, e1 in evs) / 1e3
+    dist.barrier()
+    if dist.rank == 0:
+        time.sleep(0.2)
+        sampler.stop()
+    rc, word = dit.dit_attn_gemm_check_device_error(stream)
+    if rc != 0:
+        raise RuntimeError(f"device error during the timed region: {word:#x}")
+    max_seconds = dist.max(seconds, dev)
+    value = flops * args.steps * dist.world / max_seconds / 1e12
+    achieved = flops / (seconds / args.steps) / 1e12
+
+    # End to end: the activations in from pinned host memory, Y back out, every step.
+    e2e_steps = max(3, min(args.steps, 10))
+    ha = a_cpu.view(torch.uint8).pin_memory()
+    da = torch.empty_like(a)
+    hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+
+    def e2e_step():
+        da.view(torch.uint8).copy_(ha, non_blocking=True)
+        call(da, y)
+        hy.copy_(y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = dist.max(e0.elapsed_time(e1) / 1e3, dev)
+
+    peaks, peaks_kind = load_peaks()
+    peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    clocks = sampler.summary(physical_gpu_index(dist.local_rank)) if dist.rank == 0 else {}
+    line = {
+        "metric": GEMM_FP8_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * max_seconds / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3", "data": "synthetic", "config": cfg,
+        "pct_of_peak": {"nominal_dense": 100.0 * value / dist.world / NOMINAL_TFLOPS["e4m3"],
+                        "nominal_tflops": NOMINAL_TFLOPS["e4m3"]},
+        "e2e": {"value": flops * e2e_steps * dist.world / e2e_s / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": M * K, "d2h_bytes_per_step": 2 * M * N, "steps": e2e_steps,
+                "result_matches_device": bool(torch.equal(hy, y.cpu()))},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_source": f"fp8 dense = 2 x bf16 {peaks_kind} (burst)",
+                     "traffic": profiled_traffic(w.name, kind="lowp_gemm"),
+                     "kernel": "dit_gemm::gemm_kernel<Fp8Kind> (CTA pair, persistent)", "flops_per_launch": flops},
+        "clocks": clocks,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        rate, srows, dt = gemm_oracle_rate(a_cpu[:2048], sa, w_cpu, sw, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                                "sample": f"fp64 numpy oracle (BLAS threads) on the first {srows} rows of A "
+                                          f"x [{N}, {K}]: {dt:.2f} s"}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ Ulysses FP8 payload
 
 def ulysses_degree(H: int) -> int:
@@ -1000,6 +1193,66 @@ def run_payload(args, dist: Dist):
         print(json.dumps(line), flush=True)
 
 
+PER_WORKLOAD = ["flux_1024x768", "sd35_1024_fp8", "wan_720p_81f"]
+
+
+def time_workload(w, dev, min_seconds: float = 1.0, warmup: int = 3):
+    """Device-timed attention on one workload (inputs resident, L2 flushed between
+    launches when the inputs fit in it), with its own clock record: a dict for the
+    per_workload key of the bench line."""
+    import torch
+    import attention_dit_attn_b200 as dit
+    from attention_dit_attn_b200 import workloads as wl
+    inp = wl.generate_workload(w)
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    kw = {}
+    if inp.q_scale is not None:
+        kw = dict(q_scale=inp.q_scale.to(dev).contiguous(), k_scale=inp.k_scale.to(dev).contiguous(),
+                  v_scale=inp.v_scale.to(dev).contiguous())
+    del inp
+    o = torch.empty((w.B, w.H, w.L, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    cfg = workload_config(w)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if cfg["inputs_bytes"] <= L2_BYTES \
+        else None
+    stream = torch.cuda.current_stream(dev)
+    call = lambda: dit.dit_attn_fwd(q, k, v, o, lse, scale=w.scale, stream=stream, **kw)
+    for _ in range(warmup):
+        call()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    call()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    steps = max(5, min(2000, int(min_seconds / max(a.elapsed_time(b) / 1e3, 1e-6))))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    sampler = ClockSampler()
+    sampler.start()
+    time.sleep(0.3)
+    for e0, e1 in evs:
+        if flush is not None:
+            flush.fill_(1)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    time.sleep(0.2)
+    sampler.stop()
+    rc, word = dit.dit_attn_check_device_error(stream)
+    if rc != 0:
+        raise RuntimeError(f"device error while timing {w.name}: {word:#x}")
+    sec = sum(e0.elapsed_time(e1) for e0, e1 in evs) / 1e3 / steps
+    tflops = w.flops / sec / 1e12
+    peaks, kind = load_peaks()
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak = bf16_peak if w.dtype == "bf16" else 2.0 * bf16_peak
+    return {"tflops": tflops, "ms_per_call": 1e3 * sec, "steps": steps, "dtype": w.dtype,
+            "pct_of_nominal_dense": 100.0 * tflops / NOMINAL_TFLOPS[w.dtype],
+            "frac": tflops / peak,
+            "peak_source": f"bf16 {kind} (burst)" if w.dtype == "bf16" else f"fp8 = 2 x bf16 {kind} (burst)",
+            "l2": cfg["l2"], "clocks": sampler.summary(None)}
+
+
 def run_ours(args, dist: Dist):
     import torch
     import attention_dit_attn_b200 as dit
@@ -1160,6 +1413,13 @@ def run_ours(args, dist: Dist):
     }
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
+    if dist.world == 1 and not args.no_per_workload:
+        # The other configurations, each device-timed on its own (parity cases
+        # too; reported beside the headline, not folded into it).
+        del q, k, v, o, lse, bufs, hq, hk, hv, ho, hl, inp
+        torch.cuda.empty_cache()
+        line["per_workload"] = {name: time_workload(wl.ALL[name], dev) for name in PER_WORKLOAD
+                                if name != w.name}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -1173,7 +1433,10 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["attention", "lse_merge", "residual_diff", "mxfp4_quant", "ulysses_fp8_payload"],
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="attention: skip the device timing of the other workloads (per_workload key)")
+    ap.add_argument("--op", choices=["attention", "lse_merge", "residual_diff", "mxfp4_quant", "ulysses_fp8_payload",
+                                     "gemm_fp8"],
                     default="attention")
     ap.add_argument("--parts", type=int, default=2, help="lse_merge: number of partial results (ring degree)")
     args = ap.parse_args(argv)
@@ -1188,13 +1451,14 @@ def main(argv=None):
         # The oracle runs on rank 0's host cores only; other ranks exit at once.
         if int(os.environ.get("RANK", "0")) == 0:
             {"lse_merge": run_merge_reference, "residual_diff": run_diff_reference,
-             "mxfp4_quant": run_mxfp4_reference, "ulysses_fp8_payload": run_payload_reference}.get(
+             "mxfp4_quant": run_mxfp4_reference, "ulysses_fp8_payload": run_payload_reference,
+             "gemm_fp8": run_gemm_reference}.get(
                 args.op, run_reference)(args, Dist.single())
         return
     dist = Dist(args.gpus)
     try:
         {"lse_merge": run_merge, "residual_diff": run_diff, "mxfp4_quant": run_mxfp4,
-         "ulysses_fp8_payload": run_payload}.get(
+         "ulysses_fp8_payload": run_payload, "gemm_fp8": run_gemm}.get(
             args.op, run_ours)(args, dist)
     finally:
         dist.close()

@@ -23,6 +23,12 @@
  *
  * All functions are host functions, thread-safe, and never synchronise the
  * device unless stated.  The library allocates no device memory.
+ *
+ * Every entry point runs on the current device.  One that takes device
+ * buffers checks each of them (cudaPointerGetAttributes) before anything is
+ * enqueued and returns DIT_ATTN_ERR_DEVICE when one is host memory, another
+ * GPU's memory, or covered by no CUDA allocation (dit_attn_fwd_ulysses takes
+ * peers' memory mapped into this context for its shards).
  */
 #ifndef DIT_ATTN_H
 #define DIT_ATTN_H
@@ -51,7 +57,9 @@ typedef enum {
     DIT_ATTN_ERR_ARCH = 5,     /* no CUDA device, or the current device is not sm_100 */
     DIT_ATTN_ERR_LAUNCH = 6,   /* a CUDA runtime call or the kernel launch failed */
     DIT_ATTN_ERR_TIMEOUT = 7,  /* a device-side wait ran past its time limit */
-    DIT_ATTN_ERR_VALUE = 8     /* scale is negative, NaN or infinite         */
+    DIT_ATTN_ERR_VALUE = 8,    /* scale is negative, NaN or infinite         */
+    DIT_ATTN_ERR_DEVICE = 9    /* a buffer is not device memory of the current device
+                                  (host memory, another GPU's, or no allocation) */
 } dit_attn_status;
 
 /*
@@ -76,8 +84,12 @@ typedef enum {
  *           O is vs * sum p v_hat / sum p.  Must be NULL for bf16.
  * stream    CUDA stream (0 = legacy default stream).
  *
- * Ownership: the caller owns every buffer; the library keeps no pointer
- * after the call returns (the kernel reads them in stream order).
+ * Ownership: the caller owns every buffer; the library uses no pointer
+ * after the call returns (the kernel reads them in stream order).  It keeps
+ * the TMA tensor maps of the last 16 distinct (device, q, k, v, o, B*H, L, D,
+ * dtype) calls, so a repeated call (every layer and denoising step) skips
+ * their encoding; a map holds only an address, a shape and strides, so an
+ * entry is valid for whatever buffer later sits at that address.
  * Errors: argument errors are reported before anything is enqueued.  A
  * device-side wait that exceeds its limit (default 4 s) makes the kernel
  * stop early and record an error word, reported by
@@ -325,21 +337,68 @@ int dit_attn_ulysses_check_device_error(cudaStream_t stream, uint32_t *detail);
 
 /*
  * dit_attn_residual_diff_noalloc — dit_attn_residual_diff without a caller
- * workspace and without allocating anything: the scratch is a fixed array in
- * the library's own device memory (zero at load, left zero by every call),
- * whose address is looked up once per device.  The pages have no counterpart
- * of this entry point; it exists so that a caller with no allocator at hand
- * (e.g. a captured CUDA graph built before any buffer is known) can take the
- * step-cache decision.
+ * workspace and without allocating anything.  The pages have no counterpart
+ * of this entry point.  It is for callers that cannot allocate device memory
+ * where they take the decision: a serving loop whose memory is all handed out
+ * by its own pool, which must not call cudaMalloc there (cudaMalloc can
+ * synchronise the device and stall every stream), or a host runtime that
+ * gives its plug-ins no allocator at all.
+ *
+ * The scratch is a fixed array of 16 + 16 * 1184 bytes in the library's own
+ * device memory, which every GPU that loads the library keeps until the
+ * process exits.  It is zero at load and every call leaves it zero.  Its
+ * device address is looked up (cudaGetSymbolAddress) by the first call on
+ * each device and CUDA context, with that device current; make that first
+ * call before any stream capture.  Later calls reuse the address.
  *
  * Same arguments, results and errors as dit_attn_residual_diff, minus the
  * workspace.  n above what the fixed scratch covers is rejected with
- * DIT_ATTN_ERR_SHAPE (the scratch covers every n < 2^40).  Because the scratch
- * is shared, calls on one device must be ordered (one stream, or streams
- * ordered by events); concurrent calls would race on it.
+ * DIT_ATTN_ERR_SHAPE (the scratch covers every n < 2^40).  Because every call
+ * shares the one scratch, calls on one device must be ordered (one stream, or
+ * streams ordered by events): calls that overlap on the GPU race on it.
  */
 int dit_attn_residual_diff_noalloc(const void *cur, const void *prev, long long n, float threshold,
                                    float *diff_out, int *reuse_out, cudaStream_t stream);
+
+/*
+ * dit_attn_gemm_fp8 — FP8 linear layer: y = a_scale * w_scale * (A W^T),
+ * asynchronous on `stream`.
+ *
+ * The page "How to Scale Diffusion Inference Across AMD RDNA 4 GPUs" (section
+ * "Make the Model Fit Before Tuning Latency") runs the DiT's linear layers
+ * (QKV and output projections, MLPs) in FP8; the page prints no formula, so
+ * the GEMM of the dequantised operands is taken, with one fp32
+ * dequantisation scale per tensor (x ~= s * x_hat).
+ *
+ * a   device pointer, [M, K] e4m3 codes (OCP FP8 "fn"), row-major (K
+ *     contiguous): the activations.  16-byte aligned.  Read only.
+ * w   device pointer, [N, K] e4m3 codes, row-major: the weight.  16-byte
+ *     aligned.  Read only.
+ * y   device pointer, [M, N] bf16, row-major; fully overwritten with the
+ *     fp32 result rounded to nearest.  16-byte aligned.
+ * M   rows (tokens), 0 <= M < 2^31 (0: nothing is done).
+ * N   output features, >= 8 and a multiple of 8.
+ * K   input features, >= 16 and a multiple of 16.
+ * a_scale, w_scale  finite fp32 dequantisation scales of a and w.
+ *
+ * Products are exact and accumulate in fp32 on the tensor cores
+ * (tcgen05.mma kind::f8f6f4), in a fixed order: results are deterministic.
+ * Errors (before anything is enqueued): DIT_ATTN_ERR_SHAPE, _NULL, _ALIGN,
+ * _VALUE (a non-finite scale), _ARCH, _DEVICE; DIT_ATTN_ERR_LAUNCH if the
+ * launch fails.  Device-side wait timeouts (4 s) are reported by
+ * dit_attn_gemm_check_device_error.  NaN codes are outside the contract.
+ */
+int dit_attn_gemm_fp8(const void *a, const void *w, void *y, long long M, int N, int K, float a_scale,
+                      float w_scale, cudaStream_t stream);
+
+/*
+ * dit_attn_gemm_check_device_error — dit_attn_check_device_error for the
+ * low-precision GEMM kernels (they keep their own device error word):
+ * synchronises `stream`, returns DIT_ATTN_ERR_TIMEOUT (and clears the word)
+ * if a wait of those kernels timed out, with the word in *detail if detail is
+ * non-NULL.
+ */
+int dit_attn_gemm_check_device_error(cudaStream_t stream, uint32_t *detail);
 
 #ifdef __cplusplus
 }

@@ -22,7 +22,8 @@ def test_library_exports_every_header_function(L):
                           "dit_attn_residual_diff_workspace_bytes", "dit_attn_residual_diff_noalloc",
                           "dit_attn_mxfp4_quantize", "dit_attn_block_transpose", "dit_attn_absmax_rows",
                           "dit_attn_quantize_e4m3_rows", "dit_attn_fwd_ulysses",
-                          "dit_attn_ulysses_check_device_error"}
+                          "dit_attn_ulysses_check_device_error", "dit_attn_gemm_fp8",
+                          "dit_attn_gemm_check_device_error"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -206,3 +207,23 @@ def test_require_names_the_buffer_and_its_expected_form():
     import attention_dit_attn_b200 as d
     with pytest.raises(ValueError, match="diff must be a contiguous CUDA tensor of dtype torch.float32 with 1 elements"):
         d._require(torch.zeros(1), "diff", (torch.float32,), 1)
+
+
+@pytest.mark.parametrize("args,want", [
+    ((0, 0, 0, 0, 64, 64, 1.0, 1.0), 0),          # M = 0: no-op, pointers unused
+    ((16, 16, 16, 4, 64, 24, 1.0, 1.0), 2),       # K not a multiple of 16
+    ((16, 16, 16, 4, 60, 64, 1.0, 1.0), 2),       # N not a multiple of 8
+    ((16, 0, 16, 4, 64, 64, 1.0, 1.0), 1),        # w NULL
+    ((16, 24, 16, 4, 64, 64, 1.0, 1.0), 4),       # w not 16-byte aligned
+    ((16, 16, 16, 4, 64, 64, float("nan"), 1.0), 8),   # non-finite scale
+    ((16, 16, 16, 4, 64, 64, 1.0, 1.0), 5),       # well-formed: no GPU here
+])
+def test_gemm_fp8_argument_validation(L, args, want):
+    assert dit.dit_attn_gemm_fp8_ptr(*args) == want
+
+
+def test_gemm_binding_refuses_host_buffers():
+    import attention_dit_attn_b200 as d
+    a = torch.zeros((4, 64), dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        d.dit_attn_gemm_fp8(a, a.clone(), 1.0, 1.0)

@@ -66,6 +66,22 @@ def test_fused_matches_the_oracle(cuda_lib):
     parity.check(parity.compare(o, lse, o_ref, lse_ref), "bf16")
 
 
+@pytest.mark.parametrize("n,B,H,Ls,D", [
+    (3, 1, 6, 320, 64),     # 320-row shards split 128-row tiles; last query tile partly past L
+    (3, 1, 3, 320, 128),
+    (2, 2, 4, 192, 64),
+])
+def test_fused_fp8_matches_the_oracle(cuda_lib, n, B, H, Ls, D):
+    """The FP8 fused path against the fp64 oracle on the dequantised inputs, at the
+    FP8 bound (relative Frobenius 3e-2, LSE 5e-3)."""
+    inp = wl.generate(B, H, n * Ls, D, "e4m3", seed=31 * n + Ls + D, text_rows=77, text_scale=2.0)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = _run_fused(inp, n, scale)
+    o_ref, lse_ref = parity.run_oracle(inp, scale)
+    m = parity.compare(o, lse, o_ref, lse_ref)
+    parity.check(m, "e4m3")
+
+
 def test_one_rank_writes_only_its_head_group(cuda_lib):
     inp = wl.generate(1, 8, 4 * 128, 64, "bf16", seed=9)
     o, lse = _run_fused(inp, 4, 0.125, ranks=[1])          # heads 2 and 3

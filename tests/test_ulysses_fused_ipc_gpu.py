@@ -2,7 +2,7 @@
 GPU, their shards shared through CUDA IPC, coordinated by a gloo process group
 (host barriers only: no kernel waits on another process's kernel).  The ranks'
 O and LSE shards, put together, must equal dit_attn_fwd on the whole sequence
-bit for bit."""
+bit for bit, and meet the fp64 oracle within the bf16 / FP8 bounds."""
 import datetime
 import math
 import os
@@ -74,3 +74,5 @@ def test_two_processes_share_shards_through_ipc(cuda_lib, case):
     o_ref, lse_ref = parity.run_gpu(inp, 1 / math.sqrt(D))
     assert torch.equal(o.view(torch.int16), o_ref.view(torch.int16))
     assert torch.equal(lse, lse_ref)
+    o_or, lse_or = parity.run_oracle(inp, 1 / math.sqrt(D))
+    parity.check(parity.compare(o, lse, o_or, lse_or), dtype)

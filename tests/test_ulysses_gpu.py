@@ -7,12 +7,16 @@ import os
 import socket
 import sys
 
+import numpy as np
 import pytest
 import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, os.path.join(ROOT, "tests"))
+import parity  # noqa: E402
+from oracle import e4m3_payload  # noqa: E402
 from ulysses_ref import RefOps  # noqa: E402
+from attention_dit_attn_b200 import workloads as wl  # noqa: E402
 
 pytestmark = pytest.mark.gpu
 
@@ -90,3 +94,29 @@ def test_one_rank_ulysses_equals_direct_attention(nccl_single):
     torch.cuda.synchronize()
     assert torch.equal(o8, o8_ref) and torch.equal(lse8, lse8_ref)
     assert dit.dit_attn_check_device_error()[0] == 0
+
+
+def test_one_rank_ulysses_matches_the_oracle(nccl_single):
+    """ulysses_attention against the fp64 oracle, independently of dit_attn_fwd:
+    bf16 at the bf16 bounds; with the FP8 payload, against the oracle attending
+    over the payload oracle's own quantisation of the same bf16 inputs (per-head
+    absmax, s = amax / 448, nearest-even e4m3), at the FP8 bound."""
+    from attention_dit_attn_b200.ulysses import ulysses_attention
+    B, H, L, D = 1, 4, 777, 64
+    inp = wl.generate(B, H, L, D, "bf16", seed=44, text_rows=60, text_scale=2.0)
+    q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
+    scale = 1 / math.sqrt(D)
+    o, lse = ulysses_attention(q, k, v, scale=scale)
+    o8, lse8 = ulysses_attention(q, k, v, scale=scale, fp8_comm=True)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = parity.run_oracle(inp, scale)
+    parity.check(parity.compare(o.cpu(), lse.cpu(), o_ref, lse_ref), "bf16")
+    codes, scales = [], []
+    for t in (inp.q, inp.k, inp.v):
+        x = t.to(torch.float64).numpy()
+        c, s = e4m3_payload.quantize_rows(x, e4m3_payload.absmax_rows(x, B * H))
+        codes.append(torch.from_numpy(np.ascontiguousarray(c)).view(torch.float8_e4m3fn))
+        scales.append(torch.from_numpy(s.reshape(B, H).copy()))
+    inp8 = wl.Inputs(*codes, *scales)
+    o8_ref, lse8_ref = parity.run_oracle(inp8, scale)
+    parity.check(parity.compare(o8.cpu(), lse8.cpu(), o8_ref, lse8_ref), "e4m3")
