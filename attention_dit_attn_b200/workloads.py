@@ -182,3 +182,23 @@ def gemm_operands_e4m3(M: int, N: int, K: int, seed: int = 0):
         s = float(torch.tensor(s, dtype=torch.float32))
         out += [(x / s).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn), s]
     return tuple(out)
+
+
+def gemm_operands_mxfp4(M: int, N: int, K: int, seed: int = 0, scale_spread: int = 6):
+    """MXFP4 operands drawn directly in their stored form (no conversion): packed
+    E2M1 codes, two uniform random 4-bit codes per byte (every code is a valid
+    E2M1 value, -0 included), and E8M0 block scales uniform in
+    [127 - scale_spread, 127 + scale_spread] for A and [127 - scale_spread - 4,
+    127 + scale_spread - 4] for W (smaller weights).  Layout as the quantiser
+    writes it: A codes [M, K/2], A scales [M, K/32], W codes [N, K/2],
+    W scales [N, K/32], all uint8."""
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    g = torch.Generator().manual_seed(int(seed))
+    a = torch.randint(0, 256, (M, K // 2), generator=g, dtype=torch.int32).to(torch.uint8)
+    w = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.int32).to(torch.uint8)
+    sa = torch.randint(127 - scale_spread, 127 + scale_spread + 1, (M, K // 32), generator=g,
+                       dtype=torch.int32).to(torch.uint8)
+    sw = torch.randint(123 - scale_spread, 123 + scale_spread + 1, (N, K // 32), generator=g,
+                       dtype=torch.int32).to(torch.uint8)
+    return a, sa, w, sw

@@ -277,15 +277,16 @@ def cpu_baseline(w, inp, seconds: float = 15.0):
     fifth of that), each on sampled query rows; the full call's time on this host is
     extrapolated from the all-threads rate (4*L*D FLOPs per row, B*H*L rows)."""
     import oracle
+    threads = oracle.max_threads()          # read before the one-thread run changes it
     rows, heads = plan_sample(w, inp, seconds)
-    dt, flops = oracle_sample_time(w, inp, rows, heads)
+    dt, flops = oracle_sample_time(w, inp, rows, heads, nthreads=threads)
     rate = flops / dt
-    rows1 = max(16, min(w.L, int(rows * heads * 0.2 / oracle.max_threads()) or 16))
+    rows1 = max(16, min(w.L, int(rows * heads * 0.2 / threads) or 16))
     dt1, flops1 = oracle_sample_time(w, inp, rows1, 1, nthreads=1)
-    return {"value": rate / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+    return {"value": rate / 1e12, "unit": "TFLOP/s", "cores": threads,
             "kind": "oracle",
             "sample": f"fp64 oracle on {rows} sampled query rows x {heads} head(s) of batch 0 of "
-                      f"{w.name} (all {w.L} keys per row): {dt:.1f} s on {oracle.max_threads()} threads",
+                      f"{w.name} (all {w.L} keys per row): {dt:.1f} s on {threads} threads",
             "single_thread": {"value": flops1 / dt1 / 1e12, "unit": "TFLOP/s",
                               "sample": f"{rows1} sampled query rows of head 0: {dt1:.2f} s on 1 thread"},
             "host_cpus": os.cpu_count(), "cpu_model": cpu_model(),
