@@ -29,7 +29,8 @@ __all__ = [
     "dit_attn_mxfp4_quantize", "dit_attn_mxfp4_quantize_ptr", "dit_attn_block_transpose",
     "dit_attn_absmax_rows", "dit_attn_quantize_e4m3_rows", "dit_attn_fwd_ulysses", "dit_attn_fwd_ulysses_ptr",
     "dit_attn_ulysses_check_device_error", "dit_attn_gemm_fp8", "dit_attn_gemm_fp8_ptr",
-    "dit_attn_gemm_check_device_error",
+    "dit_attn_gemm_check_device_error", "dit_attn_mxfp4_tiled_scale_bytes", "dit_attn_mxfp4_tile_scales",
+    "dit_attn_gemm_mxfp4", "dit_attn_gemm_mxfp4_ptr",
     "ensure_built", "lib",
     "header_functions", "STATUS",
 ]
@@ -106,6 +107,12 @@ def lib() -> ctypes.CDLL:
         L.dit_attn_ulysses_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.dit_attn_gemm_fp8.restype = i32
         L.dit_attn_gemm_fp8.argtypes = [vp, vp, vp, ctypes.c_longlong, i32, i32, ctypes.c_float, ctypes.c_float, vp]
+        L.dit_attn_mxfp4_tiled_scale_bytes.restype = ctypes.c_longlong
+        L.dit_attn_mxfp4_tiled_scale_bytes.argtypes = [ctypes.c_longlong, i32]
+        L.dit_attn_mxfp4_tile_scales.restype = i32
+        L.dit_attn_mxfp4_tile_scales.argtypes = [vp, vp, ctypes.c_longlong, i32, vp]
+        L.dit_attn_gemm_mxfp4.restype = i32
+        L.dit_attn_gemm_mxfp4.argtypes = [vp, vp, vp, vp, vp, ctypes.c_longlong, i32, i32, vp]
         L.dit_attn_gemm_check_device_error.restype = i32
         L.dit_attn_gemm_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         _lib = L
@@ -116,7 +123,7 @@ def header_functions() -> list[str]:
     """Names of the functions include/dit_attn.h declares."""
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(dit_attn_\w+)\s*\(", text, flags=re.M)
+    return re.findall(r"^\s*(?:const\s+)?(?:\w+\s+)*\w+\s*\**\s*(dit_attn_\w+)\s*\(", text, flags=re.M)
 
 
 def dit_attn_status_string(status: int) -> str:
@@ -555,3 +562,59 @@ def dit_attn_gemm_check_device_error(stream=None) -> tuple[int, int]:
     word = ctypes.c_uint32(0)
     rc = lib().dit_attn_gemm_check_device_error(_stream_handle(stream), ctypes.byref(word))
     return rc, word.value
+
+
+def dit_attn_mxfp4_tiled_scale_bytes(rows: int, K: int) -> int:
+    return int(lib().dit_attn_mxfp4_tiled_scale_bytes(int(rows), int(K)))
+
+
+def dit_attn_mxfp4_tile_scales(scales, K: int, tiled=None, *, stream=None):
+    """Plain [rows, K/32] E8M0 scales (uint8 CUDA tensor, as dit_attn_mxfp4_quantize writes
+    them) -> the tiled layout dit_attn_gemm_mxfp4 reads (uint8, allocated when not given)."""
+    import torch
+    _require(scales, "scales", (torch.uint8,))
+    if K % 32 or K < 32 or scales.numel() % (K // 32):
+        raise ValueError("scales must hold K/32 bytes per row, K a multiple of 32")
+    rows = scales.numel() // (K // 32)
+    nbytes = dit_attn_mxfp4_tiled_scale_bytes(rows, K)
+    if tiled is None:
+        tiled = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=scales.device)
+    _require(tiled, "tiled", (torch.uint8,))
+    if tiled.numel() < nbytes:
+        raise ValueError(f"tiled must hold {nbytes} bytes")
+    dev = _one_device(scales, tiled)
+    with torch.cuda.device(dev):
+        _check(lib().dit_attn_mxfp4_tile_scales(scales.data_ptr(), tiled.data_ptr(), rows, K,
+                                                _stream_handle(stream, dev)), "dit_attn_mxfp4_tile_scales")
+    return tiled
+
+
+def dit_attn_gemm_mxfp4_ptr(a: int, a_scales: int, w: int, w_scales: int, y: int, M: int, N: int, K: int,
+                            stream: int = 0) -> int:
+    """Raw C-ABI call with integer device pointers; returns the status code."""
+    return lib().dit_attn_gemm_mxfp4(a, a_scales, w, w_scales, y, M, N, K, stream)
+
+
+def dit_attn_gemm_mxfp4(a, a_scales_tiled, w, w_scales_tiled, y=None, *, stream=None):
+    """MXFP4 linear layer y = A W^T: a [..., K/2] and w [N, K/2] packed E2M1 codes (uint8 CUDA
+    tensors), their scales in the tiled layout (dit_attn_mxfp4_tile_scales); y bf16 [..., N]
+    (allocated when not given).  Asynchronous on ``stream``."""
+    import torch
+    for name, t in (("a", a), ("w", w), ("a_scales_tiled", a_scales_tiled), ("w_scales_tiled", w_scales_tiled)):
+        _require(t, name, (torch.uint8,))
+    if w.dim() != 2 or a.shape[-1] != w.shape[1]:
+        raise ValueError("w must be [N, K/2] with K/2 = a.shape[-1]")
+    N, K = w.shape[0], 2 * w.shape[1]
+    M = a.numel() // (K // 2) if K else 0
+    for name, t, rows in (("a_scales_tiled", a_scales_tiled, M), ("w_scales_tiled", w_scales_tiled, N)):
+        if t.numel() < dit_attn_mxfp4_tiled_scale_bytes(rows, K):
+            raise ValueError(f"{name} must hold dit_attn_mxfp4_tiled_scale_bytes({rows}, {K}) bytes")
+    if y is None:
+        y = torch.empty(tuple(a.shape[:-1]) + (N,), dtype=torch.bfloat16, device=a.device)
+    _require(y, "y", (torch.bfloat16,), M * N)
+    dev = _one_device(a, w, a_scales_tiled, w_scales_tiled, y)
+    with torch.cuda.device(dev):
+        _check(dit_attn_gemm_mxfp4_ptr(a.data_ptr(), a_scales_tiled.data_ptr(), w.data_ptr(),
+                                       w_scales_tiled.data_ptr(), y.data_ptr(), M, N, K,
+                                       _stream_handle(stream, dev)), "dit_attn_gemm_mxfp4")
+    return y

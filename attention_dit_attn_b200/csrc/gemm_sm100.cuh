@@ -89,6 +89,16 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *m, uint32_t bar, int c0, int c1,
+                                            uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, uint32_t src, int c0, int c1)
 {
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];"
@@ -387,6 +397,365 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
         __syncwarp();
         tc_fence_after();
         tmem_dealloc_pair(x.tmem, kTmemCols);
+    }
+}
+
+// ================================================================== MXFP4 (block-scaled FP4)
+//
+// Operands are MXFP4 (OCP Microscaling): packed E2M1 codes, two per byte, the
+// first element of a pair in the low nibble, and one E8M0 scale per 32
+// consecutive K elements.  The tensor core applies the scales itself
+// (tcgen05.mma kind::mxf4 block_scale scale_vec::2X: two scales per K = 64
+// MMA), reading them from TMEM.  Scales are handed to the kernel in a tiled
+// layout (dit_attn_mxfp4_tile_scales): for row r and K block b of a matrix
+// with G = 2 ceil(K / 256) four-block groups per 128-row block,
+//
+//     tiled[((r / 128) G + b / 4) 512 + 16 (r % 32) + 4 ((r % 128) / 32) + b % 4]
+//
+// so each 512-byte atom (128 rows x 4 blocks) is one contiguous bulk copy and,
+// copied to TMEM with tcgen05.cp 32x128b.warpx4 (replicated to the four lane
+// quadrants), puts the scale of row m at lane m, column base + m / 32, byte
+// b % 4, where the MMA reads it.
+//
+// One CTA (cta_group::1) owns a 128 x 256 output tile at a time: per K stage
+// of 256 elements it loads 128 rows of A and 256 of W (TMA, 128-byte swizzle)
+// and their scale atoms (bulk copies), copies the scales into a TMEM ring
+// slot and issues four MMAs of K = 64.  The epilogue reads the whole fp32
+// accumulator into registers as bf16 and hands TMEM back before it stages and
+// stores the tile, so the next tile's MMAs start while the stores drain.
+
+constexpr int kF4BM = 128, kF4BN = 256;
+constexpr int kF4Stages = 4;
+constexpr int kF4StageA = kF4BM * kBKB;            // 16 KB: 128 rows x 256 fp4
+constexpr int kF4StageB = kF4BN * kBKB;            // 32 KB
+constexpr int kF4StageSFA = 2 * 512;               // two 4-block groups of 128 rows
+constexpr int kF4StageSFB = 4 * 512;               // two groups x two 128-row blocks
+constexpr uint32_t kF4SfCols = 32;                 // TMEM columns per ring slot (8 A + 16 B used)
+constexpr uint32_t kF4TmemSf = 256;                // ring base column (accumulator: 0..255)
+
+struct F4Params {
+    int M, N, K;
+    int kb;                      // K stages of 256 elements
+    int m_tiles, n_tiles;
+    int groups;                  // G: four-block groups per 128-row block (even)
+    int w_row_blocks;            // ceil(N / 128)
+    const uint8_t *sfa;          // tiled scales of A
+    const uint8_t *sfw;          // tiled scales of W
+    unsigned long long wait_limit_ns;
+};
+
+struct F4Bars {
+    uint64_t full[kF4Stages];
+    uint64_t empty[kF4Stages];
+    uint64_t tfull;
+    uint64_t tempty;
+    uint64_t drain;
+    uint32_t tmem_base;
+    uint32_t abort;
+};
+
+struct F4Smem {
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + kF4Stages * kF4StageA;
+    static constexpr int OFF_SFA = OFF_B + kF4Stages * kF4StageB;
+    static constexpr int OFF_SFB = OFF_SFA + kF4Stages * kF4StageSFA;
+    static constexpr int OFF_O = OFF_SFB + kF4Stages * kF4StageSFB;
+    static constexpr int OFF_BAR = OFF_O + kOStage;
+    static constexpr int BYTES = OFF_BAR + 256 + 1024;
+};
+static_assert(F4Smem::BYTES <= 232448, "shared memory budget");
+
+__host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t M, uint32_t N, uint32_t sf_id)
+{
+    // [4,6) B scale id, [7,10) A format (E2M1 = 1), [10,13) B format, [17,23) N >> 3,
+    // [23] scale format (1 = E8M0), [24,29) M >> 4, [29,31) A scale id; K-major A and B.
+    return (sf_id << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24) |
+           (sf_id << 29);
+}
+
+__device__ __forceinline__ void mma_mxf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                         uint32_t sfb, uint32_t acc)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+                 ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
+                 : "memory");
+}
+
+// 32 rows x 128 bits from shared memory into TMEM lanes 0..31, replicated to
+// the four lane quadrants (4 columns).
+__device__ __forceinline__ void tmem_cp_32x128_x4(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Untiled bulk copy global -> shared, counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+struct F4Ctx {
+    F4Bars *bars;
+    uint32_t base, tmem;
+    volatile uint32_t *abort;
+    unsigned long long lim;
+    __device__ uint32_t bar(const uint64_t &b) const { return smem_u32(&b); }
+};
+
+// Scale bytes W tile n0 contributes: both 128-row blocks, or one at the end.
+__device__ __forceinline__ int f4_sfb_blocks(const F4Params &p, int n0)
+{
+    return (n0 / 128 + 1 < p.w_row_blocks) ? 2 : 1;
+}
+
+__device__ __forceinline__ void f4_producer(const F4Ctx &x, const F4Params &p, const CUtensorMap *tm_a,
+                                            const CUtensorMap *tm_w)
+{
+    const uint64_t pol_a = l2_policy_evict_first();
+    const uint64_t pol_w = l2_policy_evict_last();
+    const int tiles = p.m_tiles * p.n_tiles;
+    int it = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int m0 = (t / p.n_tiles) * kF4BM, n0 = (t % p.n_tiles) * kF4BN;
+        const int rbw = n0 / 128, nb = f4_sfb_blocks(p, n0);
+        for (int k = 0; k < p.kb; ++k, ++it) {
+            const int s = it % kF4Stages;
+            if (it >= kF4Stages &&
+                !wait_bar(x.bar(x.bars->empty[s]), ((it / kF4Stages) - 1) & 1, x.abort, x.lim, kSiteEmpty))
+                return;
+            const uint32_t full = x.bar(x.bars->full[s]);
+            mbar_arrive_expect_tx(full, kF4StageA + kF4StageB + kF4StageSFA + nb * 1024);
+            tma_load_2d(x.base + F4Smem::OFF_A + s * kF4StageA, tm_a, full, k * kBKB, m0, pol_a);
+            tma_load_2d(x.base + F4Smem::OFF_B + s * kF4StageB, tm_w, full, k * kBKB, n0, pol_w);
+            // scale atoms of groups 2k, 2k+1 (1 KB contiguous per 128-row block)
+            bulk_load(x.base + F4Smem::OFF_SFA + s * kF4StageSFA,
+                      p.sfa + ((size_t)(m0 / 128) * p.groups + 2 * k) * 512, 1024, full);
+            for (int b = 0; b < nb; ++b)
+                bulk_load(x.base + F4Smem::OFF_SFB + s * kF4StageSFB + b * 1024,
+                          p.sfw + ((size_t)(rbw + b) * p.groups + 2 * k) * 512, 1024, full);
+        }
+    }
+}
+
+__device__ __forceinline__ void f4_mma(const F4Ctx &x, const F4Params &p)
+{
+    const uint32_t base = __shfl_sync(0xffffffffu, x.base, 0);
+    const uint32_t tmem = __shfl_sync(0xffffffffu, x.tmem, 0);
+    const uint64_t a_desc = make_smem_desc(base + F4Smem::OFF_A, 16, 8 * 128, kSwizzle128B);
+    const uint64_t b_desc = make_smem_desc(base + F4Smem::OFF_B, 16, 8 * 128, kSwizzle128B);
+    // scale atoms: 32 rows of 16 bytes, no swizzle (8-row core matrices 128 bytes apart)
+    const uint64_t sfa_desc = make_smem_desc(base + F4Smem::OFF_SFA, 2048, 128, kSwizzleNone);
+    const uint64_t sfb_desc = make_smem_desc(base + F4Smem::OFF_SFB, 2048, 128, kSwizzleNone);
+    const int tiles = p.m_tiles * p.n_tiles;
+    bool ok = true;
+    int it = 0, local = 0;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
+        if (local >= 1)
+            ok = __all_sync(0xffffffffu,
+                            wait_bar(x.bar(x.bars->tempty), (local - 1) & 1, x.abort, x.lim, kSiteTmemEmpty));
+        if (!ok)
+            break;
+        tc_fence_after();
+        for (int k = 0; k < p.kb && ok; ++k, ++it) {
+            const int s = it % kF4Stages;
+            ok = __all_sync(0xffffffffu,
+                            wait_bar(x.bar(x.bars->full[s]), (it / kF4Stages) & 1, x.abort, x.lim, kSiteFull));
+            if (!ok)
+                break;
+            tc_fence_after();
+            const uint32_t sfa_t = tmem + kF4TmemSf + (uint32_t)s * kF4SfCols;
+            const uint32_t sfb_t = sfa_t + 8;
+            if (elect_one()) {
+                // A: group g -> columns sfa_t + 4g; W: group g, rows 128b.. -> sfb_t + 8g + 4b
+                for (int g = 0; g < 2; ++g) {
+                    tmem_cp_32x128_x4(sfa_t + 4 * g, sfa_desc + ((uint32_t)(s * kF4StageSFA + g * 512) >> 4));
+                    for (int b = 0; b < 2; ++b)
+                        tmem_cp_32x128_x4(sfb_t + 8 * g + 4 * b,
+                                          sfb_desc + ((uint32_t)(s * kF4StageSFB + b * 1024 + g * 512) >> 4));
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const int g = kk >> 1;
+                const uint64_t ad = a_desc + ((uint32_t)(s * kF4StageA + kk * 32) >> 4);
+                const uint64_t bd = b_desc + ((uint32_t)(s * kF4StageB + kk * 32) >> 4);
+                if (elect_one())
+                    mma_mxf4(tmem, ad, bd, idesc_mxf4(kF4BM, kF4BN, (uint32_t)(kk & 1) * 2u), sfa_t + 4 * g,
+                             sfb_t + 8 * g, (k > 0 || kk > 0) ? 1u : 0u);
+            }
+            if (elect_one())
+                mma_commit(x.bar(x.bars->empty[s]));
+            __syncwarp();
+        }
+        if (ok && elect_one())
+            mma_commit(x.bar(x.bars->tfull));
+        __syncwarp();
+    }
+    if (!ok) {
+        if (elect_one())
+            mma_commit(x.bar(x.bars->drain));
+        __syncwarp();
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(x.bar(x.bars->drain), 0) && globaltimer_ns() - t0 < 50000000ull) {
+        }
+    }
+}
+
+// Epilogue: thread r owns row m0 + r (TMEM lane r).  All 256 accumulator
+// columns go to registers as bf16 pairs, TMEM is handed back, then the tile is
+// staged one 64-column box at a time and stored with TMA (clipped at M, N).
+__device__ __forceinline__ void f4_epilogue(const F4Ctx &x, const F4Params &p, const CUtensorMap *tm_y, int warp,
+                                            int lane)
+{
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const bool issuer = warp == kEpiWarp0 && lane == 0;
+    const int tiles = p.m_tiles * p.n_tiles;
+    bool ok = true;
+    int local = 0;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
+        const int m0 = (t / p.n_tiles) * kF4BM, n0 = (t % p.n_tiles) * kF4BN;
+        ok = __all_sync(0xffffffffu, wait_bar(x.bar(x.bars->tfull), local & 1, x.abort, x.lim, kSiteTmemFull));
+        if (!bar_and(1, 128, ok)) {
+            ok = false;
+            break;
+        }
+        tc_fence_after();
+        uint32_t pk[128];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t v[32];
+            tmem_ld32(x.tmem + lane_off + 32 * c, v);
+            tmem_wait_ld_regs(v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                pk[16 * c + i] = *reinterpret_cast<uint32_t *>(&h);
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(x.bar(x.bars->tempty));
+#pragma unroll
+        for (int c = 0; c < kF4BN / kOBox; ++c) {
+            if (n0 + c * kOBox >= p.N)
+                break;                                   // uniform over the 128 threads
+            // the single staging box: the previous store must have read it
+            if (issuer)
+                bulk_wait_group_read<0>();
+            named_bar(1, 128);
+            const uint32_t st = x.base + F4Smem::OFF_O;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint32_t off = (uint32_t)row * 128u + (uint32_t)ch * 16u;
+                const uint32_t swz_off = off ^ ((off >> 3) & 0x70u);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(st + swz_off), "r"(pk[32 * c + 4 * ch]),
+                             "r"(pk[32 * c + 4 * ch + 1]), "r"(pk[32 * c + 4 * ch + 2]), "r"(pk[32 * c + 4 * ch + 3])
+                             : "memory");
+            }
+            fence_proxy_async_smem();
+            named_bar(1, 128);
+            if (issuer) {
+                tma_store_2d(tm_y, st, n0 + c * kOBox, m0);
+                bulk_commit_group();
+            }
+        }
+    }
+    if (issuer)
+        bulk_wait_group_all();
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
+                 const __grid_constant__ CUtensorMap tm_y, const F4Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    F4Bars *bars = reinterpret_cast<F4Bars *>(smem_raw + (base - raw_addr) + F4Smem::OFF_BAR);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kF4Stages; ++s) {
+            mbar_init(smem_u32(&bars->full[s]), 1);
+            mbar_init(smem_u32(&bars->empty[s]), 1);
+        }
+        mbar_init(smem_u32(&bars->tfull), 1);
+        mbar_init(smem_u32(&bars->tempty), 4);           // the 4 epilogue warps
+        mbar_init(smem_u32(&bars->drain), 1);
+        bars->abort = 0u;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_a);
+        tma_prefetch_desc(&tm_w);
+        tma_prefetch_desc(&tm_y);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    F4Ctx x;
+    x.bars = bars;
+    x.base = base;
+    x.tmem = bars->tmem_base;
+    x.abort = &bars->abort;
+    x.lim = p.wait_limit_ns;
+
+    if (warp == 0) {
+        if (lane == 0)
+            f4_producer(x, p, &tm_a, &tm_w);
+    } else if (warp == 1) {
+        f4_mma(x, p);
+    } else {
+        f4_epilogue(x, p, &tm_y, warp, lane);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(x.tmem, kTmemCols);
+    }
+}
+
+// Scale tiling: plain [rows, K / 32] E8M0 bytes -> the tiled layout above
+// (zero where the padded rows or blocks have no scale).  One thread per
+// 16-byte chunk of the output: one row's 4 blocks for 4 rows 32 apart.
+__global__ void tile_scales_kernel(const uint8_t *__restrict__ plain, uint32_t *__restrict__ tiled, int rows,
+                                   int kblocks, int groups, long long chunks)
+{
+    for (long long c = blockIdx.x * (long long)blockDim.x + threadIdx.x; c < chunks;
+         c += (long long)gridDim.x * blockDim.x) {
+        const long long atom = c >> 5;                   // 32 chunks of 16 bytes per atom
+        const int r32 = (int)(c & 31);
+        const int g = (int)(atom % groups);
+        const long long rb = atom / groups;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const long long r = rb * 128 + q * 32 + r32;
+            uint32_t v = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int kb = g * 4 + b;
+                if (r < rows && kb < kblocks)
+                    v |= (uint32_t)plain[r * kblocks + kb] << (8 * b);
+            }
+            w[q] = v;
+        }
+        reinterpret_cast<uint4 *>(tiled)[c] = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 

@@ -20,6 +20,7 @@ constexpr unsigned long long kWaitLimitNs = 4000000000ull;
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sms[kMaxDevices];
 std::atomic<int> g_attr_set[kMaxDevices];
+std::atomic<int> g_attr_set_f4[kMaxDevices];
 
 PFN_cuTensorMapEncodeTiled_v12000 encoder()
 {
@@ -138,6 +139,98 @@ int dit_attn_gemm_fp8(const void *a, const void *w, void *y, long long M, int N,
     p.out_scale = a_scale * w_scale;
     p.wait_limit_ns = kWaitLimitNs;
     return launch<dit_gemm::Fp8Kind>(ta, tw, ty, p, device, stream);
+}
+
+long long dit_attn_mxfp4_tiled_scale_bytes(long long rows, int K)
+{
+    if (rows < 1 || K < 32 || K % 32 != 0)
+        return 0;
+    const long long row_blocks = (rows + 127) / 128;
+    const long long groups = 2 * ((K + 255) / 256);
+    return row_blocks * groups * 512;
+}
+
+int dit_attn_mxfp4_tile_scales(const void *plain, void *tiled, long long rows, int K, cudaStream_t stream)
+{
+    if (rows < 0 || K < 32 || K % 32 != 0 || rows > 0x7FFFFFFFll)
+        return DIT_ATTN_ERR_SHAPE;
+    if (rows == 0)
+        return DIT_ATTN_OK;
+    if (plain == nullptr || tiled == nullptr)
+        return DIT_ATTN_ERR_NULL;
+    if (!dit_abi::aligned(tiled, 16))
+        return DIT_ATTN_ERR_ALIGN;
+    int device = 0;
+    const int rc = check_device(&device);
+    if (rc != DIT_ATTN_OK)
+        return rc;
+    if (!dit_abi::device_buffers(device, {plain, tiled}))
+        return DIT_ATTN_ERR_DEVICE;
+    const long long chunks = dit_attn_mxfp4_tiled_scale_bytes(rows, K) / 16;
+    const int groups = 2 * ((K + 255) / 256);
+    const long long blocks = (chunks + 255) / 256;
+    dit_gemm::tile_scales_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(
+        static_cast<const uint8_t *>(plain), static_cast<uint32_t *>(tiled), (int)rows, K / 32, groups, chunks);
+    return cudaGetLastError() == cudaSuccess ? DIT_ATTN_OK : DIT_ATTN_ERR_LAUNCH;
+}
+
+int dit_attn_gemm_mxfp4(const void *a, const void *a_scales, const void *w, const void *w_scales, void *y,
+                        long long M, int N, int K, cudaStream_t stream)
+{
+    if (M < 0 || N < 8 || N % 8 != 0 || K < 32 || K % 32 != 0 || M > 0x7FFFFFFFll)
+        return DIT_ATTN_ERR_SHAPE;
+    if (M == 0)
+        return DIT_ATTN_OK;
+    if (a == nullptr || w == nullptr || y == nullptr || a_scales == nullptr || w_scales == nullptr)
+        return DIT_ATTN_ERR_NULL;
+    if (!dit_abi::aligned(a, 16) || !dit_abi::aligned(w, 16) || !dit_abi::aligned(y, 16) ||
+        !dit_abi::aligned(a_scales, 16) || !dit_abi::aligned(w_scales, 16))
+        return DIT_ATTN_ERR_ALIGN;
+    int device = 0;
+    const int rc = check_device(&device);
+    if (rc != DIT_ATTN_OK)
+        return rc;
+    if (!dit_abi::device_buffers(device, {a, w, y, a_scales, w_scales}))
+        return DIT_ATTN_ERR_DEVICE;
+    auto kern = dit_gemm::gemm_mxf4_kernel;
+    if (g_attr_set_f4[device].load(std::memory_order_acquire) == 0) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dit_gemm::F4Smem::BYTES) !=
+            cudaSuccess)
+            return DIT_ATTN_ERR_LAUNCH;
+        g_attr_set_f4[device].store(1, std::memory_order_release);
+    }
+    int sms = g_sms[device].load(std::memory_order_relaxed);
+    if (sms == 0) {
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+            return DIT_ATTN_ERR_LAUNCH;
+        g_sms[device].store(sms, std::memory_order_relaxed);
+    }
+    CUtensorMap ta, tw, ty;
+    if (!make_map_2d(&ta, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, M, K / 2, dit_gemm::kBKB, dit_gemm::kF4BM) ||
+        !make_map_2d(&tw, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, dit_gemm::kBKB, dit_gemm::kF4BN) ||
+        !make_map_2d(&ty, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, 2ll * N, dit_gemm::kOBox, dit_gemm::kF4BM))
+        return DIT_ATTN_ERR_LAUNCH;
+    dit_gemm::F4Params p{};
+    p.M = (int)M;
+    p.N = N;
+    p.K = K;
+    p.groups = 2 * ((K + 255) / 256);
+    p.kb = p.groups / 2;
+    p.m_tiles = (int)((M + dit_gemm::kF4BM - 1) / dit_gemm::kF4BM);
+    p.n_tiles = (N + dit_gemm::kF4BN - 1) / dit_gemm::kF4BN;
+    p.w_row_blocks = (N + 127) / 128;
+    p.sfa = static_cast<const uint8_t *>(a_scales);
+    p.sfw = static_cast<const uint8_t *>(w_scales);
+    p.wait_limit_ns = kWaitLimitNs;
+    const long long tiles = (long long)p.m_tiles * p.n_tiles;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles < sms ? tiles : sms));
+    cfg.blockDim = dim3(dit_gemm::kThreads);
+    cfg.dynamicSmemBytes = dit_gemm::F4Smem::BYTES;
+    cfg.stream = stream;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tw, ty, p) != cudaSuccess)
+        return DIT_ATTN_ERR_LAUNCH;
+    return cudaGetLastError() == cudaSuccess ? DIT_ATTN_OK : DIT_ATTN_ERR_LAUNCH;
 }
 
 int dit_attn_gemm_check_device_error(cudaStream_t stream, uint32_t *detail)

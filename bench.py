@@ -33,6 +33,9 @@ hot path is one kernel launch).  Prints ONE JSON line on rank 0.
 * --op gemm_fp8: the FP8 linear layer Y = A W^T of the workload's projection
   (M = B*L tokens, N = K = H*D features), e4m3 in, bf16 out; TFLOP/s,
   roofline against the fp8 dense peak (2 x the measured bf16 peak).
+* --op gemm_mxfp4: the same projection in MXFP4 (E2M1 codes, one E8M0 scale per
+  32 K elements), roofline against the fp4 dense peak (4 x the measured bf16
+  peak).
 * --op ulysses_fp8_payload: the per-GPU preparation of Ulysses' FP8 all-to-all
   payload for one [B, H, L, D] bf16 tensor of the workload: per-head absmax,
   e4m3 quantisation, heads grouped by destination rank; GB/s of algorithmic
@@ -61,10 +64,13 @@ MERGE_METRIC = "LSE merge of partial attentions: GB/s of algorithmic HBM traffic
 DIFF_METRIC = "step-cache residual-change decision: GB/s of algorithmic HBM traffic at 1 GPU"
 MXFP4_METRIC = "MXFP4 1x32 activation quantiser: GB/s of algorithmic HBM traffic at 1 GPU"
 GEMM_FP8_METRIC = "FP8 linear layer Y = A W^T (e4m3 in, bf16 out): TFLOP/s at 1 GPU"
+GEMM_MXFP4_METRIC = "MXFP4 linear layer Y = A W^T (block-scaled E2M1 in, bf16 out): TFLOP/s at 1 GPU"
 PAYLOAD_METRIC = ("Ulysses FP8 payload preparation (absmax, e4m3 quantise, head grouping): "
                   "GB/s of algorithmic HBM traffic at 1 GPU")
 DEFAULT_WORKLOAD = "flux_2048_cfg"      # the first workload with L >= 16k (the stated target)
-NOMINAL_TFLOPS = {"bf16": 2250.0, "e4m3": 4500.0}
+NOMINAL_TFLOPS = {"bf16": 2250.0, "e4m3": 4500.0, "e2m1": 9000.0}
+# Dense tensor rate of each input type relative to bf16 (nominal B200 figures: 2.25 / 4.5 / 9 PFLOP/s).
+RATE_VS_BF16 = {"bf16": 1.0, "e4m3": 2.0, "e2m1": 4.0}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 L2_BYTES = 126 * 1024 * 1024
 
@@ -88,7 +94,8 @@ KERNEL_SOURCES = {
     "residual_diff": ["residual_diff.cu"],
     "mxfp4_quant": ["mxfp4_quant.cu"],
     "ulysses_ops": ["ulysses_ops.cu"],
-    "lowp_gemm": ["gemm_sm100.cuh", "lowp_gemm.cu", "sm100_ptx.cuh"],
+    "lowp_gemm_fp8": ["gemm_sm100.cuh", "lowp_gemm.cu", "sm100_ptx.cuh"],
+    "lowp_gemm_mxfp4": ["gemm_sm100.cuh", "lowp_gemm.cu", "sm100_ptx.cuh"],
 }
 
 
@@ -849,9 +856,13 @@ def gemm_shape(w):
     return w.B * w.L, w.H * w.D, w.H * w.D
 
 
-def gemm_config(w, M, N, K):
-    in_bytes = M * K + N * K
-    return {"workload": w.name, "op": "gemm_fp8", "M": M, "N": N, "K": K, "input_dtype": "e4m3",
+def gemm_config(w, M, N, K, kind="fp8"):
+    if kind == "fp8":
+        in_bytes = M * K + N * K
+    else:
+        in_bytes = (M + N) * (K // 2 + K // 32)
+    return {"workload": w.name, "op": "gemm_" + kind, "M": M, "N": N, "K": K,
+            "input_dtype": "e4m3" if kind == "fp8" else "MXFP4 (E2M1 + E8M0 per 32)",
             "output_dtype": "bf16", "flops_per_call": 2.0 * M * N * K,
             "bytes_per_call": in_bytes + 2 * M * N,
             "l2": "inputs and output larger than L2" if in_bytes + 2 * M * N > L2_BYTES
@@ -859,38 +870,51 @@ def gemm_config(w, M, N, K):
             "parallelism": "replicas"}
 
 
-def gemm_oracle_rate(a, sa, w_, sw, seconds: float):
+def gemm_oracle_rate(a, sa, w_, sw, seconds: float, kind="fp8"):
     """fp64 oracle (oracle/lowp_gemm.py) on the first rows of A: (TFLOP/s, rows, s)."""
     import torch
     from oracle import lowp_gemm
     ac, wc = a.view(torch.uint8).numpy(), w_.view(torch.uint8).numpy()
+    K = wc.shape[1] if kind == "fp8" else 2 * wc.shape[1]
     rows = 4
     while True:
         t0 = time.perf_counter()
-        lowp_gemm.gemm_e4m3(ac[:rows], sa, wc, sw)
+        if kind == "fp8":
+            lowp_gemm.gemm_e4m3(ac[:rows], sa, wc, sw)
+        else:
+            lowp_gemm.gemm_mxfp4(ac[:rows], sa[:rows].numpy(), wc, sw.numpy())
         dt = time.perf_counter() - t0
         if dt >= seconds / 4 or rows >= ac.shape[0]:
-            return 2.0 * rows * wc.shape[0] * wc.shape[1] / dt / 1e12, rows, dt
+            return 2.0 * rows * wc.shape[0] * K / dt / 1e12, rows, dt
         rows = min(ac.shape[0], rows * 4)
+
+
+def gemm_operands(w, M, N, K, kind):
+    from attention_dit_attn_b200 import workloads as wl
+    if kind == "fp8":
+        return wl.gemm_operands_e4m3(M, N, K, seed=w.seed)
+    return wl.gemm_operands_mxfp4(M, N, K, seed=w.seed)
 
 
 def run_gemm_reference(args, dist: Dist):
     if dist.rank != 0:
         return
     from attention_dit_attn_b200 import workloads as wl
+    kind = args.op.split("_")[1]
     w = wl.ALL[args.workload]
     M, N, K = gemm_shape(w)
-    a, sa, w_, sw = wl.gemm_operands_e4m3(min(M, 1024), N, K, seed=w.seed)
+    a, sa, w_, sw = gemm_operands(w, min(M, 1024), N, K, kind)
     per = 60.0 / max(1, args.steps + args.warmup)
     for _ in range(args.warmup):
-        gemm_oracle_rate(a, sa, w_, sw, per)
-    rates = [gemm_oracle_rate(a, sa, w_, sw, per) for _ in range(args.steps)]
+        gemm_oracle_rate(a, sa, w_, sw, per, kind)
+    rates = [gemm_oracle_rate(a, sa, w_, sw, per, kind) for _ in range(args.steps)]
     value = statistics.median(r[0] for r in rates)
     line = {
-        "impl": "reference", "metric": GEMM_FP8_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": GEMM_FP8_METRIC if kind == "fp8" else GEMM_MXFP4_METRIC, "value": value,
+        "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * 2.0 * M * N * K / (value * 1e12),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": gemm_config(w, M, N, K),
+        "data": "synthetic", "config": gemm_config(w, M, N, K, kind),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
                          "sample": f"each step: fp64 numpy oracle (BLAS) on {rates[0][1]} rows of A x [{N}, {K}]"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -907,18 +931,28 @@ def run_gemm(args, dist: Dist):
     dit.ensure_built()
     torch.cuda.set_device(dist.local_rank)
     dev = torch.device("cuda", dist.local_rank)
+    kind = args.op.split("_")[1]                       # fp8 | mxfp4
     w = wl.ALL[args.workload]
     M, N, K = gemm_shape(w)
-    a_cpu, sa, w_cpu, sw = wl.gemm_operands_e4m3(M, N, K, seed=w.seed)
+    a_cpu, sa, w_cpu, sw = gemm_operands(w, M, N, K, kind)
     a, wt = a_cpu.to(dev), w_cpu.to(dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    cfg = gemm_config(w, M, N, K)
+    stream = torch.cuda.current_stream(dev)
+    if kind == "fp8":
+        call = lambda aa, yy: dit.dit_attn_gemm_fp8(aa, wt, sa, sw, y=yy, stream=stream)
+        dtype, kern = "e4m3", "dit_gemm::gemm_kernel<Fp8Kind> (CTA pair, persistent)"
+    else:
+        # Scales in the tiled layout the tensor cores read: the weight's once,
+        # the activation's as part of each end-to-end step.
+        ta = dit.dit_attn_mxfp4_tile_scales(sa.to(dev), K)
+        tw = dit.dit_attn_mxfp4_tile_scales(sw.to(dev), K)
+        call = lambda aa, yy: dit.dit_attn_gemm_mxfp4(aa, ta, wt, tw, y=yy, stream=stream)
+        dtype, kern = "e2m1", "dit_gemm::gemm_mxf4_kernel (one CTA per SM, persistent)"
+    cfg = gemm_config(w, M, N, K, kind)
     flops = cfg["flops_per_call"]
     flush = None
     if cfg["bytes_per_call"] <= L2_BYTES:
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    call = lambda aa, yy: dit.dit_attn_gemm_fp8(aa, wt, sa, sw, y=yy, stream=stream)
     for _ in range(args.warmup):
         call(a, y)
     torch.cuda.synchronize(dev)
@@ -952,15 +986,25 @@ def run_gemm(args, dist: Dist):
     value = flops * args.steps * dist.world / max_seconds / 1e12
     achieved = flops / (seconds / args.steps) / 1e12
 
-    # End to end: the activations in from pinned host memory, Y back out, every step.
+    # End to end: the activations (and MXFP4 scales) in from pinned host memory, Y back
+    # out, every step.
     e2e_steps = max(3, min(args.steps, 10))
     ha = a_cpu.view(torch.uint8).pin_memory()
     da = torch.empty_like(a)
     hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    if kind == "mxfp4":
+        hs = sa.pin_memory()
+        ds = torch.empty_like(hs, device=dev)
+        dta = torch.empty_like(ta)
 
     def e2e_step():
         da.view(torch.uint8).copy_(ha, non_blocking=True)
-        call(da, y)
+        if kind == "fp8":
+            call(da, y)
+        else:
+            ds.copy_(hs, non_blocking=True)
+            dit.dit_attn_mxfp4_tile_scales(ds, K, tiled=dta, stream=stream)
+            dit.dit_attn_gemm_mxfp4(da, dta, wt, tw, y=y, stream=stream)
         hy.copy_(y, non_blocking=True)
 
     e2e_step()
@@ -973,29 +1017,34 @@ def run_gemm(args, dist: Dist):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_s = dist.max(e0.elapsed_time(e1) / 1e3, dev)
+    h2d = ha.numel() + (hs.numel() if kind == "mxfp4" else 0)
 
     peaks, peaks_kind = load_peaks()
-    peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak = RATE_VS_BF16[dtype] * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     clocks = sampler.summary(physical_gpu_index(dist.local_rank)) if dist.rank == 0 else {}
     line = {
-        "metric": GEMM_FP8_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": dist.world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * max_seconds / args.steps,
+        "metric": GEMM_FP8_METRIC if kind == "fp8" else GEMM_MXFP4_METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * max_seconds / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3", "data": "synthetic", "config": cfg,
-        "pct_of_peak": {"nominal_dense": 100.0 * value / dist.world / NOMINAL_TFLOPS["e4m3"],
-                        "nominal_tflops": NOMINAL_TFLOPS["e4m3"]},
+        "dtype": dtype, "data": "synthetic", "config": cfg,
+        "pct_of_peak": {"nominal_dense": 100.0 * value / dist.world / NOMINAL_TFLOPS[dtype],
+                        "nominal_tflops": NOMINAL_TFLOPS[dtype]},
         "e2e": {"value": flops * e2e_steps * dist.world / e2e_s / 1e12, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": M * K, "d2h_bytes_per_step": 2 * M * N, "steps": e2e_steps,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 2 * M * N, "steps": e2e_steps,
                 "result_matches_device": bool(torch.equal(hy, y.cpu()))},
         "gpu_launches": args.steps,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "peak_source": f"fp8 dense = 2 x bf16 {peaks_kind} (burst)",
-                     "traffic": profiled_traffic(w.name, kind="lowp_gemm"),
-                     "kernel": "dit_gemm::gemm_kernel<Fp8Kind> (CTA pair, persistent)", "flops_per_launch": flops},
+                     "frac": achieved / peak,
+                     "peak_source": f"{dtype} dense = {RATE_VS_BF16[dtype]:g} x bf16 {peaks_kind} (burst), "
+                                    "the nominal dense-rate ratio",
+                     "traffic": profiled_traffic(w.name, kind="lowp_gemm_" + kind),
+                     "kernel": kern, "flops_per_launch": flops},
         "clocks": clocks,
     }
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        rate, srows, dt = gemm_oracle_rate(a_cpu[:2048], sa, w_cpu, sw, args.cpu_seconds)
+        rate, srows, dt = gemm_oracle_rate(a_cpu[:2048], sa if kind == "fp8" else sa[:2048], w_cpu, sw,
+                                           args.cpu_seconds, kind)
         line["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
                                 "sample": f"fp64 numpy oracle (BLAS threads) on the first {srows} rows of A "
                                           f"x [{N}, {K}]: {dt:.2f} s"}
@@ -1437,7 +1486,7 @@ def main(argv=None):
     ap.add_argument("--no-per-workload", action="store_true",
                     help="attention: skip the device timing of the other workloads (per_workload key)")
     ap.add_argument("--op", choices=["attention", "lse_merge", "residual_diff", "mxfp4_quant", "ulysses_fp8_payload",
-                                     "gemm_fp8"],
+                                     "gemm_fp8", "gemm_mxfp4"],
                     default="attention")
     ap.add_argument("--parts", type=int, default=2, help="lse_merge: number of partial results (ring degree)")
     args = ap.parse_args(argv)
@@ -1453,13 +1502,13 @@ def main(argv=None):
         if int(os.environ.get("RANK", "0")) == 0:
             {"lse_merge": run_merge_reference, "residual_diff": run_diff_reference,
              "mxfp4_quant": run_mxfp4_reference, "ulysses_fp8_payload": run_payload_reference,
-             "gemm_fp8": run_gemm_reference}.get(
+             "gemm_fp8": run_gemm_reference, "gemm_mxfp4": run_gemm_reference}.get(
                 args.op, run_reference)(args, Dist.single())
         return
     dist = Dist(args.gpus)
     try:
         {"lse_merge": run_merge, "residual_diff": run_diff, "mxfp4_quant": run_mxfp4,
-         "ulysses_fp8_payload": run_payload, "gemm_fp8": run_gemm}.get(
+         "ulysses_fp8_payload": run_payload, "gemm_fp8": run_gemm, "gemm_mxfp4": run_gemm}.get(
             args.op, run_ours)(args, dist)
     finally:
         dist.close()

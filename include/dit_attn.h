@@ -392,6 +392,69 @@ int dit_attn_gemm_fp8(const void *a, const void *w, void *y, long long M, int N,
                       float w_scale, cudaStream_t stream);
 
 /*
+ * dit_attn_mxfp4_tiled_scale_bytes — size in bytes of the tiled E8M0 scale
+ * layout dit_attn_gemm_mxfp4 reads, for a matrix of `rows` rows and K columns
+ * (K a multiple of 32): ceil(rows / 128) * G * 512 with G = 2 ceil(K / 256).
+ * Returns 0 for rows < 1 or a bad K.  Host only; no CUDA call.
+ */
+long long dit_attn_mxfp4_tiled_scale_bytes(long long rows, int K);
+
+/*
+ * dit_attn_mxfp4_tile_scales — rearranges MXFP4 block scales from the plain
+ * layout dit_attn_mxfp4_quantize writes ([rows, K / 32] E8M0 bytes, row-major)
+ * into the tiled layout the tensor cores read in dit_attn_gemm_mxfp4:
+ *
+ *     tiled[((r / 128) G + b / 4) 512 + 16 (r % 32) + 4 ((r % 128) / 32) + b % 4]
+ *         = plain[r][b],   G = 2 ceil(K / 256),
+ *
+ * zero for the padding rows and blocks.  Each 512-byte atom holds the scales
+ * of 128 rows for 4 consecutive 32-element blocks.  This layout is this
+ * library's choice (the pages say nothing of scale layouts); it is the one
+ * from which a bulk copy and a TMEM copy put every scale where the block-scaled
+ * MMA reads it.  Weights are tiled once; activations after each quantisation.
+ *
+ * plain  device pointer, [rows, K / 32] bytes.  Read only.
+ * tiled  device pointer, dit_attn_mxfp4_tiled_scale_bytes(rows, K) bytes,
+ *        16-byte aligned.  Fully overwritten.
+ * Errors (before anything is enqueued): DIT_ATTN_ERR_SHAPE, _NULL, _ALIGN,
+ * _ARCH, _DEVICE; DIT_ATTN_ERR_LAUNCH.  rows = 0 is a no-op.
+ */
+int dit_attn_mxfp4_tile_scales(const void *plain, void *tiled, long long rows, int K, cudaStream_t stream);
+
+/*
+ * dit_attn_gemm_mxfp4 — MXFP4 linear layer: Y = A W^T with A and W in MXFP4
+ * (OCP Microscaling: E2M1 values sharing one E8M0 scale per 32 consecutive K
+ * elements), bf16 out, asynchronous on `stream`.
+ *
+ * The page "Accelerating Diffusers and xDiT Image Generation with MXFP4 using
+ * AMD Quark on AMD Instinct MI350 GPUs" (sections "MXFP4 Quantization" and
+ * "MXFP4 Kernel") runs the DiT's linear layers as FP4 x FP4 GEMMs on MXFP4
+ * activations (quantised on the fly in 1x32 blocks, dit_attn_mxfp4_quantize)
+ * and MXFP4 weights.  The page prints no formula; this computes the GEMM of
+ * the dequantised operands, y[m][n] = sum_k a[m][k] w[n][k].
+ *
+ * a         device pointer, [M, K / 2] packed E2M1 codes (two per byte, the
+ *           first element of a pair in the low nibble), 16-byte aligned.
+ * a_scales  device pointer, A's scales in the tiled layout
+ *           (dit_attn_mxfp4_tile_scales), 16-byte aligned.
+ * w         device pointer, [N, K / 2] packed codes of the weight.
+ * w_scales  device pointer, W's scales, tiled.
+ * y         device pointer, [M, N] bf16 row-major; fully overwritten with the
+ *           fp32 result rounded to nearest.  16-byte aligned.
+ * M >= 0 (0: nothing is done), N >= 8 and a multiple of 8, K >= 32 and a
+ * multiple of 32.
+ *
+ * The scaled products are exact and accumulate in fp32 on the tensor cores
+ * (tcgen05.mma kind::mxf4, block scales read from TMEM), in a fixed order.
+ * Errors (before anything is enqueued): DIT_ATTN_ERR_SHAPE, _NULL, _ALIGN,
+ * _ARCH, _DEVICE; DIT_ATTN_ERR_LAUNCH.  Device-side wait timeouts are
+ * reported by dit_attn_gemm_check_device_error.  E8M0 0xFF (NaN) scales are
+ * outside the contract.
+ */
+int dit_attn_gemm_mxfp4(const void *a, const void *a_scales, const void *w, const void *w_scales, void *y,
+                        long long M, int N, int K, cudaStream_t stream);
+
+/*
  * dit_attn_gemm_check_device_error — dit_attn_check_device_error for the
  * low-precision GEMM kernels (they keep their own device error word):
  * synchronises `stream`, returns DIT_ATTN_ERR_TIMEOUT (and clears the word)

@@ -23,7 +23,8 @@ def test_library_exports_every_header_function(L):
                           "dit_attn_mxfp4_quantize", "dit_attn_block_transpose", "dit_attn_absmax_rows",
                           "dit_attn_quantize_e4m3_rows", "dit_attn_fwd_ulysses",
                           "dit_attn_ulysses_check_device_error", "dit_attn_gemm_fp8",
-                          "dit_attn_gemm_check_device_error"}
+                          "dit_attn_gemm_check_device_error", "dit_attn_mxfp4_tiled_scale_bytes",
+                          "dit_attn_mxfp4_tile_scales", "dit_attn_gemm_mxfp4"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -227,3 +228,30 @@ def test_gemm_binding_refuses_host_buffers():
     a = torch.zeros((4, 64), dtype=torch.uint8)
     with pytest.raises(ValueError):
         d.dit_attn_gemm_fp8(a, a.clone(), 1.0, 1.0)
+
+
+def test_mxfp4_tiled_scale_bytes(L):
+    import attention_dit_attn_b200 as d
+    assert d.dit_attn_mxfp4_tiled_scale_bytes(1, 32) == 1 * 2 * 512
+    assert d.dit_attn_mxfp4_tiled_scale_bytes(128, 256) == 1 * 2 * 512
+    assert d.dit_attn_mxfp4_tiled_scale_bytes(129, 288) == 2 * 4 * 512
+    assert d.dit_attn_mxfp4_tiled_scale_bytes(33792, 3072) == 264 * 24 * 512
+    assert d.dit_attn_mxfp4_tiled_scale_bytes(0, 64) == 0
+    assert d.dit_attn_mxfp4_tiled_scale_bytes(4, 48) == 0
+
+
+def test_gemm_mxfp4_argument_validation(L):
+    call = dit.dit_attn_gemm_mxfp4_ptr
+    assert call(0, 0, 0, 0, 0, 0, 64, 64) == 0                 # M = 0: no-op
+    assert call(16, 16, 16, 16, 16, 4, 64, 48) == 2            # K not a multiple of 32
+    assert call(16, 16, 16, 16, 16, 4, 60, 64) == 2            # N not a multiple of 8
+    assert call(16, 0, 16, 16, 16, 4, 64, 64) == 1             # a_scales NULL
+    assert call(16, 24, 16, 16, 16, 4, 64, 64) == 4            # a_scales not 16-byte aligned
+    assert call(16, 16, 16, 16, 16, 4, 64, 64) == 5            # well-formed: no GPU here
+    L.dit_attn_mxfp4_tile_scales.restype = ctypes.c_int
+    L.dit_attn_mxfp4_tile_scales.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int,
+                                             ctypes.c_void_p]
+    assert L.dit_attn_mxfp4_tile_scales(16, 16, 4, 48, None) == 2
+    assert L.dit_attn_mxfp4_tile_scales(None, None, 0, 64, None) == 0
+    assert L.dit_attn_mxfp4_tile_scales(16, 24, 4, 64, None) == 4
+    assert L.dit_attn_mxfp4_tile_scales(16, 16, 4, 64, None) == 5
