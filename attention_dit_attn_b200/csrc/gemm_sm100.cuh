@@ -99,10 +99,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *m, 
         : "memory");
 }
 
+// The output is written once and read by nobody in this kernel: it goes to L2
+// with the evict-first policy, so it does not push out the operand tiles.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, uint32_t src, int c0, int c1)
 {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];"
-                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(src), "r"(c0), "r"(c1)
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;"
+                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(src), "r"(c0), "r"(c1), "l"(pol)
                  : "memory");
 }
 
@@ -182,7 +186,8 @@ template <class Kind>
 __device__ __forceinline__ void producer(const Ctx &x, const GemmParams &p, const CUtensorMap *tm_a,
                                          const CUtensorMap *tm_w)
 {
-    const uint64_t pol_a = l2_policy_evict_first();
+    // A block: read by the n_tiles pairs that work on it side by side; W: by every pair.
+    const uint64_t pol_a = l2_policy_evict_last();
     const uint64_t pol_w = l2_policy_evict_last();
     const bool leader = x.rank == 0;
     const int tiles = p.m_tiles * p.n_tiles;
@@ -514,7 +519,7 @@ __device__ __forceinline__ int f4_sfb_blocks(const F4Params &p, int n0)
 __device__ __forceinline__ void f4_producer(const F4Ctx &x, const F4Params &p, const CUtensorMap *tm_a,
                                             const CUtensorMap *tm_w)
 {
-    const uint64_t pol_a = l2_policy_evict_first();
+    const uint64_t pol_a = l2_policy_evict_last();
     const uint64_t pol_w = l2_policy_evict_last();
     const int tiles = p.m_tiles * p.n_tiles;
     int it = 0;
