@@ -219,9 +219,12 @@ __device__ __forceinline__ void pair_producer(const PairCtx<C> &x, const FwdPara
         }
     }
     if (!ok) {
-        // Give copies already in flight time to land before the cluster exits.
+        // Give copies already in flight time to land before the cluster exits:
+        // 1 ms, far above the latency of a tile load from this GPU's memory or
+        // over NVLink from a peer's (a few microseconds).  Only the abort path
+        // (after a wait has run out of time) pays it.
         const uint64_t t0 = globaltimer_ns();
-        while (globaltimer_ns() - t0 < 20000ull) {
+        while (globaltimer_ns() - t0 < 1000000ull) {
         }
     }
 }

@@ -422,53 +422,27 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
 // quadrants), puts the scale of row m at lane m, column base + m / 32, byte
 // b % 4, where the MMA reads it.
 //
-// One CTA (cta_group::1) owns a 128 x 256 output tile at a time: per K stage
-// of 256 elements it loads 128 rows of A and 256 of W (TMA, 128-byte swizzle)
-// and their scale atoms (bulk copies), copies the scales into a TMEM ring
-// slot and issues four MMAs of K = 64.  The epilogue reads the whole fp32
-// accumulator into registers as bf16 and hands TMEM back before it stages and
-// stores the tile, so the next tile's MMAs start while the stores drain.
+// The kernel (gemm_mxf4_pair_kernel, below) runs on CTA pairs.  Per K stage of
+// 256 elements each CTA loads its share of A and W and their scale atoms,
+// the leader copies the scales into a TMEM ring slot and issues four MMAs of
+// K = 64.  The epilogue reads the whole fp32 accumulator into registers as
+// bf16 and hands TMEM back before it stages and stores the tile, so the next
+// tile's MMAs start while the stores drain.
 
 constexpr int kF4BM = 128, kF4BN = 256;
-constexpr int kF4Stages = 4;
-constexpr int kF4StageA = kF4BM * kBKB;            // 16 KB: 128 rows x 256 fp4
-constexpr int kF4StageB = kF4BN * kBKB;            // 32 KB
-constexpr int kF4StageSFA = 2 * 512;               // two 4-block groups of 128 rows
-constexpr int kF4StageSFB = 4 * 512;               // two groups x two 128-row blocks
 constexpr uint32_t kF4SfCols = 32;                 // TMEM columns per ring slot (8 A + 16 B used)
 constexpr uint32_t kF4TmemSf = 256;                // ring base column (accumulator: 0..255)
 
 struct F4Params {
     int M, N, K;
     int kb;                      // K stages of 256 elements
-    int m_tiles, n_tiles;
+    int m_tiles, n_tiles;        // ceil(M / 256), ceil(N / 256)
     int groups;                  // G: four-block groups per 128-row block (even)
     int w_row_blocks;            // ceil(N / 128)
     const uint8_t *sfa;          // tiled scales of A
     const uint8_t *sfw;          // tiled scales of W
     unsigned long long wait_limit_ns;
 };
-
-struct F4Bars {
-    uint64_t full[kF4Stages];
-    uint64_t empty[kF4Stages];
-    uint64_t tfull;
-    uint64_t tempty;
-    uint64_t drain;
-    uint32_t tmem_base;
-    uint32_t abort;
-};
-
-struct F4Smem {
-    static constexpr int OFF_A = 0;
-    static constexpr int OFF_B = OFF_A + kF4Stages * kF4StageA;
-    static constexpr int OFF_SFA = OFF_B + kF4Stages * kF4StageB;
-    static constexpr int OFF_SFB = OFF_SFA + kF4Stages * kF4StageSFA;
-    static constexpr int OFF_O = OFF_SFB + kF4Stages * kF4StageSFB;
-    static constexpr int OFF_BAR = OFF_O + kOStage;
-    static constexpr int BYTES = OFF_BAR + 256 + 1024;
-};
-static_assert(F4Smem::BYTES <= 232448, "shared memory budget");
 
 __host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t M, uint32_t N, uint32_t sf_id)
 {
@@ -478,86 +452,121 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t M, uint32_t N, uint32
            (sf_id << 29);
 }
 
-__device__ __forceinline__ void mma_mxf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
-                                         uint32_t sfb, uint32_t acc)
+
+// ------------------------------------------------------------------ MXFP4 on CTA pairs
+//
+// The same GEMM on CTA pairs (cta_group::2): a pair owns a 256 x 256 tile,
+// each CTA loads its 128 rows of A and 128 of the tile's 256 rows of W per K
+// stage, so each SM streams half the W tile through shared memory, and the
+// leader issues M = N = 256 block-scaled MMAs.  Scales, measured with a
+// probe: tcgen05.cp with cta_group::2 (issued once by the leader) copies each
+// CTA's own shared memory into its own TMEM, and each CTA's half of the MMA
+// reads A's scales for its own 128 rows and W's scales for all 256 columns
+// from its own TMEM.  So each CTA loads the scale atoms of its A rows and of
+// both 128-row blocks of the W tile.  The atoms come as plain 2-D TMA boxes
+// (4 rows of 256 bytes = two 512-byte atoms) over the tiled array, so both
+// CTAs' copies count on the leader's barrier; a W block past N is out of
+// range and TMA fills it with zeros (finite scales).
+
+constexpr int kP4Stages = 5;
+constexpr int kP4StageA = kF4BM * kBKB;           // 16 KB: this CTA's 128 rows of A
+constexpr int kP4StageB = (kF4BN / 2) * kBKB;     // 16 KB: this CTA's 128 rows of W
+constexpr int kP4StageSFA = 1024, kP4StageSFB = 2048;
+constexpr int kP4StageBytes = kP4StageA + kP4StageB + kP4StageSFA + kP4StageSFB;
+
+struct P4Bars {
+    uint64_t full[kP4Stages];   // leader: stage s of both CTAs landed
+    uint64_t empty[kP4Stages];  // each CTA: the MMAs reading stage s completed
+    uint64_t tfull;             // each CTA: the accumulator holds a finished tile
+    uint64_t tempty;            // leader: both CTAs' epilogues have read it
+    uint64_t drain;
+    uint32_t tmem_base;
+    uint32_t abort;
+};
+
+struct P4Smem {
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + kP4Stages * kP4StageA;
+    static constexpr int OFF_SFA = OFF_B + kP4Stages * kP4StageB;
+    static constexpr int OFF_SFB = OFF_SFA + kP4Stages * kP4StageSFA;
+    static constexpr int OFF_O = OFF_SFB + kP4Stages * kP4StageSFB;
+    static constexpr int OFF_BAR = OFF_O + kOStage;
+    static constexpr int BYTES = OFF_BAR + 256 + 1024;
+};
+static_assert(P4Smem::BYTES <= 232448, "shared memory budget");
+static_assert(kF4TmemSf + kP4Stages * kF4SfCols <= kTmemCols, "TMEM budget");
+
+__device__ __forceinline__ void mma2_mxf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                          uint32_t sfb, uint32_t acc)
 {
     asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+                 "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
                  ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
                  : "memory");
 }
 
-// 32 rows x 128 bits from shared memory into TMEM lanes 0..31, replicated to
-// the four lane quadrants (4 columns).
-__device__ __forceinline__ void tmem_cp_32x128_x4(uint32_t taddr, uint64_t sdesc)
+// Each CTA's 32 x 128-bit shared-memory block into its own TMEM (issued by the leader).
+__device__ __forceinline__ void tmem_cp2_32x128_x4(uint32_t taddr, uint64_t sdesc)
 {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-// Untiled bulk copy global -> shared, counted in bytes on `bar`.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-
-struct F4Ctx {
-    F4Bars *bars;
-    uint32_t base, tmem;
+struct P4Ctx {
+    P4Bars *bars;
+    uint32_t base, tmem, rank;
     volatile uint32_t *abort;
     unsigned long long lim;
     __device__ uint32_t bar(const uint64_t &b) const { return smem_u32(&b); }
+    __device__ uint32_t leader_bar(const uint64_t &b) const { return mapa_shared(smem_u32(&b), 0); }
 };
 
-// Scale bytes W tile n0 contributes: both 128-row blocks, or one at the end.
-__device__ __forceinline__ int f4_sfb_blocks(const F4Params &p, int n0)
-{
-    return (n0 / 128 + 1 < p.w_row_blocks) ? 2 : 1;
-}
-
-__device__ __forceinline__ void f4_producer(const F4Ctx &x, const F4Params &p, const CUtensorMap *tm_a,
-                                            const CUtensorMap *tm_w)
+__device__ __forceinline__ void p4_producer(const P4Ctx &x, const F4Params &p, const CUtensorMap *tm_a,
+                                            const CUtensorMap *tm_w, const CUtensorMap *tm_sa,
+                                            const CUtensorMap *tm_sw)
 {
     const uint64_t pol_a = l2_policy_evict_last();
     const uint64_t pol_w = l2_policy_evict_last();
+    const bool leader = x.rank == 0;
     const int tiles = p.m_tiles * p.n_tiles;
     int it = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-        const int m0 = (t / p.n_tiles) * kF4BM, n0 = (t % p.n_tiles) * kF4BN;
-        const int rbw = n0 / 128, nb = f4_sfb_blocks(p, n0);
+    for (int t = blockIdx.x / 2; t < tiles; t += gridDim.x / 2) {
+        const int m0 = (t / p.n_tiles) * 2 * kF4BM, n0 = (t % p.n_tiles) * kF4BN;
+        const int rba = m0 / 128 + (int)x.rank, rbw = n0 / 128;
         for (int k = 0; k < p.kb; ++k, ++it) {
-            const int s = it % kF4Stages;
-            if (it >= kF4Stages &&
-                !wait_bar(x.bar(x.bars->empty[s]), ((it / kF4Stages) - 1) & 1, x.abort, x.lim, kSiteEmpty))
+            const int s = it % kP4Stages;
+            if (it >= kP4Stages &&
+                !wait_bar(x.bar(x.bars->empty[s]), ((it / kP4Stages) - 1) & 1, x.abort, x.lim, kSiteEmpty))
                 return;
-            const uint32_t full = x.bar(x.bars->full[s]);
-            mbar_arrive_expect_tx(full, kF4StageA + kF4StageB + kF4StageSFA + nb * 1024);
-            tma_load_2d(x.base + F4Smem::OFF_A + s * kF4StageA, tm_a, full, k * kBKB, m0, pol_a);
-            tma_load_2d(x.base + F4Smem::OFF_B + s * kF4StageB, tm_w, full, k * kBKB, n0, pol_w);
-            // scale atoms of groups 2k, 2k+1 (1 KB contiguous per 128-row block)
-            bulk_load(x.base + F4Smem::OFF_SFA + s * kF4StageSFA,
-                      p.sfa + ((size_t)(m0 / 128) * p.groups + 2 * k) * 512, 1024, full);
-            for (int b = 0; b < nb; ++b)
-                bulk_load(x.base + F4Smem::OFF_SFB + s * kF4StageSFB + b * 1024,
-                          p.sfw + ((size_t)(rbw + b) * p.groups + 2 * k) * 512, 1024, full);
+            if (leader)
+                mbar_arrive_expect_tx(x.bar(x.bars->full[s]), 2 * kP4StageBytes);
+            const uint32_t full = x.leader_bar(x.bars->full[s]);
+            tma_load_2d_pair(x.base + P4Smem::OFF_A + s * kP4StageA, tm_a, full, k * kBKB, m0 + (int)x.rank * kF4BM,
+                             pol_a);
+            tma_load_2d_pair(x.base + P4Smem::OFF_B + s * kP4StageB, tm_w, full, k * kBKB,
+                             n0 + (int)x.rank * (kF4BN / 2), pol_w);
+            // scale atoms of groups 2k, 2k+1: 4 rows of 256 bytes from (block * G + 2k) * 2
+            tma_load_2d_pair(x.base + P4Smem::OFF_SFA + s * kP4StageSFA, tm_sa, full, 0, (rba * p.groups + 2 * k) * 2,
+                             pol_a);
+            for (int b = 0; b < 2; ++b)
+                tma_load_2d_pair(x.base + P4Smem::OFF_SFB + s * kP4StageSFB + b * 1024, tm_sw, full, 0,
+                                 ((rbw + b) * p.groups + 2 * k) * 2, pol_w);
         }
     }
 }
 
-__device__ __forceinline__ void f4_mma(const F4Ctx &x, const F4Params &p)
+__device__ __forceinline__ void p4_mma(const P4Ctx &x, const F4Params &p)
 {
+    constexpr uint16_t kBoth = 0x3;
     const uint32_t base = __shfl_sync(0xffffffffu, x.base, 0);
     const uint32_t tmem = __shfl_sync(0xffffffffu, x.tmem, 0);
-    const uint64_t a_desc = make_smem_desc(base + F4Smem::OFF_A, 16, 8 * 128, kSwizzle128B);
-    const uint64_t b_desc = make_smem_desc(base + F4Smem::OFF_B, 16, 8 * 128, kSwizzle128B);
-    // scale atoms: 32 rows of 16 bytes, no swizzle (8-row core matrices 128 bytes apart)
-    const uint64_t sfa_desc = make_smem_desc(base + F4Smem::OFF_SFA, 2048, 128, kSwizzleNone);
-    const uint64_t sfb_desc = make_smem_desc(base + F4Smem::OFF_SFB, 2048, 128, kSwizzleNone);
+    const uint64_t a_desc = make_smem_desc(base + P4Smem::OFF_A, 16, 8 * 128, kSwizzle128B);
+    const uint64_t b_desc = make_smem_desc(base + P4Smem::OFF_B, 16, 8 * 128, kSwizzle128B);
+    const uint64_t sfa_desc = make_smem_desc(base + P4Smem::OFF_SFA, 2048, 128, kSwizzleNone);
+    const uint64_t sfb_desc = make_smem_desc(base + P4Smem::OFF_SFB, 2048, 128, kSwizzleNone);
     const int tiles = p.m_tiles * p.n_tiles;
     bool ok = true;
     int it = 0, local = 0;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
+    for (int t = blockIdx.x / 2; t < tiles && ok; t += gridDim.x / 2, ++local) {
         if (local >= 1)
             ok = __all_sync(0xffffffffu,
                             wait_bar(x.bar(x.bars->tempty), (local - 1) & 1, x.abort, x.lim, kSiteTmemEmpty));
@@ -565,44 +574,43 @@ __device__ __forceinline__ void f4_mma(const F4Ctx &x, const F4Params &p)
             break;
         tc_fence_after();
         for (int k = 0; k < p.kb && ok; ++k, ++it) {
-            const int s = it % kF4Stages;
+            const int s = it % kP4Stages;
             ok = __all_sync(0xffffffffu,
-                            wait_bar(x.bar(x.bars->full[s]), (it / kF4Stages) & 1, x.abort, x.lim, kSiteFull));
+                            wait_bar(x.bar(x.bars->full[s]), (it / kP4Stages) & 1, x.abort, x.lim, kSiteFull));
             if (!ok)
                 break;
             tc_fence_after();
             const uint32_t sfa_t = tmem + kF4TmemSf + (uint32_t)s * kF4SfCols;
             const uint32_t sfb_t = sfa_t + 8;
             if (elect_one()) {
-                // A: group g -> columns sfa_t + 4g; W: group g, rows 128b.. -> sfb_t + 8g + 4b
                 for (int g = 0; g < 2; ++g) {
-                    tmem_cp_32x128_x4(sfa_t + 4 * g, sfa_desc + ((uint32_t)(s * kF4StageSFA + g * 512) >> 4));
+                    tmem_cp2_32x128_x4(sfa_t + 4 * g, sfa_desc + ((uint32_t)(s * kP4StageSFA + g * 512) >> 4));
                     for (int b = 0; b < 2; ++b)
-                        tmem_cp_32x128_x4(sfb_t + 8 * g + 4 * b,
-                                          sfb_desc + ((uint32_t)(s * kF4StageSFB + b * 1024 + g * 512) >> 4));
+                        tmem_cp2_32x128_x4(sfb_t + 8 * g + 4 * b,
+                                           sfb_desc + ((uint32_t)(s * kP4StageSFB + b * 1024 + g * 512) >> 4));
                 }
             }
             __syncwarp();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const int g = kk >> 1;
-                const uint64_t ad = a_desc + ((uint32_t)(s * kF4StageA + kk * 32) >> 4);
-                const uint64_t bd = b_desc + ((uint32_t)(s * kF4StageB + kk * 32) >> 4);
+                const uint64_t ad = a_desc + ((uint32_t)(s * kP4StageA + kk * 32) >> 4);
+                const uint64_t bd = b_desc + ((uint32_t)(s * kP4StageB + kk * 32) >> 4);
                 if (elect_one())
-                    mma_mxf4(tmem, ad, bd, idesc_mxf4(kF4BM, kF4BN, (uint32_t)(kk & 1) * 2u), sfa_t + 4 * g,
-                             sfb_t + 8 * g, (k > 0 || kk > 0) ? 1u : 0u);
+                    mma2_mxf4(tmem, ad, bd, idesc_mxf4(2 * kF4BM, kF4BN, (uint32_t)(kk & 1) * 2u), sfa_t + 4 * g,
+                              sfb_t + 8 * g, (k > 0 || kk > 0) ? 1u : 0u);
             }
             if (elect_one())
-                mma_commit(x.bar(x.bars->empty[s]));
+                mma2_commit_mc(x.bar(x.bars->empty[s]), kBoth);
             __syncwarp();
         }
         if (ok && elect_one())
-            mma_commit(x.bar(x.bars->tfull));
+            mma2_commit_mc(x.bar(x.bars->tfull), kBoth);
         __syncwarp();
     }
     if (!ok) {
         if (elect_one())
-            mma_commit(x.bar(x.bars->drain));
+            mma2_commit(x.bar(x.bars->drain));
         __syncwarp();
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(x.bar(x.bars->drain), 0) && globaltimer_ns() - t0 < 50000000ull) {
@@ -610,10 +618,7 @@ __device__ __forceinline__ void f4_mma(const F4Ctx &x, const F4Params &p)
     }
 }
 
-// Epilogue: thread r owns row m0 + r (TMEM lane r).  All 256 accumulator
-// columns go to registers as bf16 pairs, TMEM is handed back, then the tile is
-// staged one 64-column box at a time and stored with TMA (clipped at M, N).
-__device__ __forceinline__ void f4_epilogue(const F4Ctx &x, const F4Params &p, const CUtensorMap *tm_y, int warp,
+__device__ __forceinline__ void p4_epilogue(const P4Ctx &x, const F4Params &p, const CUtensorMap *tm_y, int warp,
                                             int lane)
 {
     const int quad = warp & 3;
@@ -621,10 +626,11 @@ __device__ __forceinline__ void f4_epilogue(const F4Ctx &x, const F4Params &p, c
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const bool issuer = warp == kEpiWarp0 && lane == 0;
     const int tiles = p.m_tiles * p.n_tiles;
+    const uint32_t tempty_leader = x.leader_bar(x.bars->tempty);
     bool ok = true;
     int local = 0;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
-        const int m0 = (t / p.n_tiles) * kF4BM, n0 = (t % p.n_tiles) * kF4BN;
+    for (int t = blockIdx.x / 2; t < tiles && ok; t += gridDim.x / 2, ++local) {
+        const int m0 = (t / p.n_tiles) * 2 * kF4BM + (int)x.rank * kF4BM, n0 = (t % p.n_tiles) * kF4BN;
         ok = __all_sync(0xffffffffu, wait_bar(x.bar(x.bars->tfull), local & 1, x.abort, x.lim, kSiteTmemFull));
         if (!bar_and(1, 128, ok)) {
             ok = false;
@@ -646,16 +652,15 @@ __device__ __forceinline__ void f4_epilogue(const F4Ctx &x, const F4Params &p, c
         tc_fence_before();
         __syncwarp();
         if (lane == 0)
-            mbar_arrive(x.bar(x.bars->tempty));
+            mbar_arrive_cluster(tempty_leader);
 #pragma unroll
         for (int c = 0; c < kF4BN / kOBox; ++c) {
             if (n0 + c * kOBox >= p.N)
-                break;                                   // uniform over the 128 threads
-            // the single staging box: the previous store must have read it
+                break;
             if (issuer)
                 bulk_wait_group_read<0>();
             named_bar(1, 128);
-            const uint32_t st = x.base + F4Smem::OFF_O;
+            const uint32_t st = x.base + P4Smem::OFF_O;
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
                 const uint32_t off = (uint32_t)row * 128u + (uint32_t)ch * 16u;
@@ -677,22 +682,24 @@ __device__ __forceinline__ void f4_epilogue(const F4Ctx &x, const F4Params &p, c
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
-                 const __grid_constant__ CUtensorMap tm_y, const F4Params p)
+gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
+                      const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_sa,
+                      const __grid_constant__ CUtensorMap tm_sw, const F4Params p)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
-    F4Bars *bars = reinterpret_cast<F4Bars *>(smem_raw + (base - raw_addr) + F4Smem::OFF_BAR);
+    P4Bars *bars = reinterpret_cast<P4Bars *>(smem_raw + (base - raw_addr) + P4Smem::OFF_BAR);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kF4Stages; ++s) {
+        for (int s = 0; s < kP4Stages; ++s) {
             mbar_init(smem_u32(&bars->full[s]), 1);
             mbar_init(smem_u32(&bars->empty[s]), 1);
         }
         mbar_init(smem_u32(&bars->tfull), 1);
-        mbar_init(smem_u32(&bars->tempty), 4);           // the 4 epilogue warps
+        mbar_init(smem_u32(&bars->tempty), 8);           // 4 epilogue warps x 2 CTAs
         mbar_init(smem_u32(&bars->drain), 1);
         bars->abort = 0u;
         fence_barrier_init();
@@ -702,36 +709,42 @@ gemm_mxf4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
         tma_prefetch_desc(&tm_a);
         tma_prefetch_desc(&tm_w);
         tma_prefetch_desc(&tm_y);
+        tma_prefetch_desc(&tm_sa);
+        tma_prefetch_desc(&tm_sw);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_u32(&bars->tmem_base), kTmemCols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
 
-    F4Ctx x;
+    P4Ctx x;
     x.bars = bars;
     x.base = base;
     x.tmem = bars->tmem_base;
+    x.rank = rank;
     x.abort = &bars->abort;
     x.lim = p.wait_limit_ns;
 
     if (warp == 0) {
         if (lane == 0)
-            f4_producer(x, p, &tm_a, &tm_w);
+            p4_producer(x, p, &tm_a, &tm_w, &tm_sa, &tm_sw);
     } else if (warp == 1) {
-        f4_mma(x, p);
+        if (rank == 0)
+            p4_mma(x, p);
     } else {
-        f4_epilogue(x, p, &tm_y, warp, lane);
+        p4_epilogue(x, p, &tm_y, warp, lane);
     }
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     if (warp == 1) {
+        __syncwarp();
         tc_fence_after();
-        tmem_dealloc(x.tmem, kTmemCols);
+        tmem_dealloc_pair(x.tmem, kTmemCols);
     }
 }
 

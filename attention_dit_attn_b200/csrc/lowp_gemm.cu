@@ -37,9 +37,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder()
 }
 
 // 2-D map over a row-major [rows, row_bytes] byte matrix (or bf16 with elt 2):
-// dims (cols, rows), box (box_cols, box_rows), 128-byte swizzle.
+// dims (cols, rows), box (box_cols, box_rows), 128-byte swizzle unless told otherwise.
 bool make_map_2d(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, long long cols, long long rows,
-                 long long row_bytes, int box_cols, int box_rows)
+                 long long row_bytes, int box_cols, int box_rows,
+                 CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B)
 {
     auto enc = encoder();
     if (!enc)
@@ -48,9 +49,8 @@ bool make_map_2d(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, long l
     const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
     const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1u, 1u};
-    return enc(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return enc(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int check_device(int *device)
@@ -192,9 +192,9 @@ int dit_attn_gemm_mxfp4(const void *a, const void *a_scales, const void *w, cons
         return rc;
     if (!dit_abi::device_buffers(device, {a, w, y, a_scales, w_scales}))
         return DIT_ATTN_ERR_DEVICE;
-    auto kern = dit_gemm::gemm_mxf4_kernel;
+    auto kern = dit_gemm::gemm_mxf4_pair_kernel;
     if (g_attr_set_f4[device].load(std::memory_order_acquire) == 0) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dit_gemm::F4Smem::BYTES) !=
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dit_gemm::P4Smem::BYTES) !=
             cudaSuccess)
             return DIT_ATTN_ERR_LAUNCH;
         g_attr_set_f4[device].store(1, std::memory_order_release);
@@ -205,30 +205,45 @@ int dit_attn_gemm_mxfp4(const void *a, const void *a_scales, const void *w, cons
             return DIT_ATTN_ERR_LAUNCH;
         g_sms[device].store(sms, std::memory_order_relaxed);
     }
-    CUtensorMap ta, tw, ty;
-    if (!make_map_2d(&ta, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, M, K / 2, dit_gemm::kBKB, dit_gemm::kF4BM) ||
-        !make_map_2d(&tw, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, dit_gemm::kBKB, dit_gemm::kF4BN) ||
-        !make_map_2d(&ty, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, 2ll * N, dit_gemm::kOBox, dit_gemm::kF4BM))
-        return DIT_ATTN_ERR_LAUNCH;
     dit_gemm::F4Params p{};
     p.M = (int)M;
     p.N = N;
     p.K = K;
     p.groups = 2 * ((K + 255) / 256);
     p.kb = p.groups / 2;
-    p.m_tiles = (int)((M + dit_gemm::kF4BM - 1) / dit_gemm::kF4BM);
+    p.m_tiles = (int)((M + 2 * dit_gemm::kF4BM - 1) / (2 * dit_gemm::kF4BM));
     p.n_tiles = (N + dit_gemm::kF4BN - 1) / dit_gemm::kF4BN;
     p.w_row_blocks = (N + 127) / 128;
     p.sfa = static_cast<const uint8_t *>(a_scales);
     p.sfw = static_cast<const uint8_t *>(w_scales);
     p.wait_limit_ns = kWaitLimitNs;
+    // Scale atoms as 256-byte rows: two rows per 512-byte atom.
+    const long long sa_rows = dit_attn_mxfp4_tiled_scale_bytes(M, K) / 256;
+    const long long sw_rows = dit_attn_mxfp4_tiled_scale_bytes(N, K) / 256;
+    CUtensorMap ta, tw, ty, tsa, tsw;
+    if (!make_map_2d(&ta, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, M, K / 2, dit_gemm::kBKB, dit_gemm::kF4BM) ||
+        !make_map_2d(&tw, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, dit_gemm::kBKB, dit_gemm::kF4BN / 2) ||
+        !make_map_2d(&ty, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, 2ll * N, dit_gemm::kOBox, dit_gemm::kF4BM) ||
+        !make_map_2d(&tsa, a_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 256, sa_rows, 256, 256, 4,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_2d(&tsw, w_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 256, sw_rows, 256, 256, 4,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+        return DIT_ATTN_ERR_LAUNCH;
     const long long tiles = (long long)p.m_tiles * p.n_tiles;
+    const long long clusters = tiles < sms / 2 ? tiles : sms / 2;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(tiles < sms ? tiles : sms));
+    cfg.gridDim = dim3((unsigned)(2 * clusters));
     cfg.blockDim = dim3(dit_gemm::kThreads);
-    cfg.dynamicSmemBytes = dit_gemm::F4Smem::BYTES;
+    cfg.dynamicSmemBytes = dit_gemm::P4Smem::BYTES;
     cfg.stream = stream;
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tw, ty, p) != cudaSuccess)
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tw, ty, tsa, tsw, p) != cudaSuccess)
         return DIT_ATTN_ERR_LAUNCH;
     return cudaGetLastError() == cudaSuccess ? DIT_ATTN_OK : DIT_ATTN_ERR_LAUNCH;
 }
