@@ -133,8 +133,33 @@ def dit_attn_status_string(status: int) -> str:
 def _stream_handle(stream, device=None) -> int:
     import torch
     if stream is None:
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        if raw is not None:
+            # The raw handle of torch's current stream, without building a Stream object.
+            index = device.index if device is not None and device.index is not None else torch.cuda.current_device()
+            return int(raw(index))
         stream = torch.cuda.current_stream(device)
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class _Nothing:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+_NOTHING = _Nothing()
+
+
+def _on_device(dev):
+    """Context that makes ``dev`` current: a no-op when it already is (the common
+    case, and a few microseconds less per call)."""
+    import torch
+    if dev.index is None or dev.index == torch.cuda.current_device():
+        return _NOTHING
+    return torch.cuda.device(dev)
 
 
 def _one_device(*tensors):
@@ -201,7 +226,7 @@ def dit_attn_fwd(q, k, v, o=None, lse=None, *, scale: float | None = None, q_sca
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     dev = _one_device(q, k, v, o, lse, q_scale, k_scale, v_scale)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         rc = dit_attn_fwd_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                               None if lse is None else lse.data_ptr(), B, H, L, D, float(scale), dtype,
                               *scales, stream=_stream_handle(stream, dev))
@@ -270,7 +295,7 @@ def dit_attn_lse_merge(parts, o=None, lse=None, *, want_lse: bool = True, stream
                               or not lse.is_contiguous() or not lse.is_cuda):
         raise ValueError("lse must be a contiguous fp32 CUDA tensor with one value per row")
     dev = _one_device(o, lse, *[t for part in parts for t in part])
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         rc = dit_attn_lse_merge_ptr([oc.data_ptr() for oc, _ in parts], [lc.data_ptr() for _, lc in parts],
                                     o.data_ptr(), None if lse is None else lse.data_ptr(), rows, D,
                                     _stream_handle(stream, dev))
@@ -318,7 +343,7 @@ def dit_attn_residual_diff(cur, prev, threshold: float = 0.12, *, workspace=None
     _require(diff, "diff", (torch.float32,), 1)
     _require(reuse, "reuse", (torch.int32,), 1)
     dev = _one_device(cur, prev, workspace, diff, reuse)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         rc = dit_attn_residual_diff_ptr(cur.data_ptr(), prev.data_ptr(), n, float(threshold),
                                         workspace.data_ptr(), workspace.numel(), diff.data_ptr(), reuse.data_ptr(),
                                         _stream_handle(stream, dev))
@@ -344,7 +369,7 @@ def dit_attn_residual_diff_noalloc(cur, prev, threshold: float = 0.12, *, diff=N
     _require(diff, "diff", (torch.float32,), 1)
     _require(reuse, "reuse", (torch.int32,), 1)
     dev = _one_device(cur, prev, diff, reuse)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         rc = lib().dit_attn_residual_diff_noalloc(cur.data_ptr(), prev.data_ptr(), cur.numel(),
                                                   ctypes.c_float(threshold), diff.data_ptr(), reuse.data_ptr(),
                                                   _stream_handle(stream, dev))
@@ -375,7 +400,7 @@ def dit_attn_mxfp4_quantize(x, q=None, scales=None, *, stream=None):
         if not (t.is_cuda and t.dtype == torch.uint8 and t.is_contiguous() and t.numel() == rows * cols):
             raise ValueError(f"{name} must be a contiguous uint8 CUDA tensor with {rows * cols} elements")
     dev = _one_device(x, q, scales)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         rc = dit_attn_mxfp4_quantize_ptr(x.data_ptr(), q.data_ptr(), scales.data_ptr(), rows, K,
                                          _stream_handle(stream, dev))
     if rc != 0:
@@ -416,7 +441,7 @@ def dit_attn_block_transpose(x, R: int, C: int, out=None, *, stream=None):
         out = torch.empty_like(x)
     _require(out, "out", nbytes=nbytes)
     dev = _one_device(x, out)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(lib().dit_attn_block_transpose(x.data_ptr(), out.data_ptr(), R, C, nbytes // (R * C),
                                               _stream_handle(stream, dev)), "dit_attn_block_transpose")
     return out
@@ -433,7 +458,7 @@ def dit_attn_absmax_rows(x, rows: int, out=None, *, stream=None):
         out = torch.empty(rows, dtype=torch.float32, device=x.device)
     _require(out, "out", (torch.float32,), rows)
     dev = _one_device(x, out)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(lib().dit_attn_absmax_rows(x.data_ptr(), out.data_ptr(), rows, x.numel() // max(rows, 1),
                                           _stream_handle(stream, dev)), "dit_attn_absmax_rows")
     return out
@@ -456,7 +481,7 @@ def dit_attn_quantize_e4m3_rows(x, amax, q=None, scale=None, *, stream=None):
     _require(q, "q", (torch.float8_e4m3fn, torch.uint8), x.numel())
     _require(scale, "scale", (torch.float32,), rows)
     dev = _one_device(x, amax, q, scale)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(lib().dit_attn_quantize_e4m3_rows(x.data_ptr(), amax.data_ptr(), q.data_ptr(), scale.data_ptr(),
                                                  rows, x.numel() // max(rows, 1), _stream_handle(stream, dev)),
                "dit_attn_quantize_e4m3_rows")
@@ -516,7 +541,7 @@ def dit_attn_fwd_ulysses(q_shards, k_shards, v_shards, o_shards, lse_shards=None
     own = [q_shards[rank], k_shards[rank], v_shards[rank], o_shards[rank]]
     dev = _one_device(*own, None if lse_shards is None else lse_shards[rank], q_scale, k_scale, v_scale)
     ptrs = lambda ts: [t.data_ptr() for t in ts]
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         rc = dit_attn_fwd_ulysses_ptr(ptrs(q_shards), ptrs(k_shards), ptrs(v_shards), ptrs(o_shards),
                                       None if lse_shards is None else ptrs(lse_shards), rank, B, H, Ls, D,
                                       float(scale), dtype, *scales, stream=_stream_handle(stream, dev))
@@ -551,7 +576,7 @@ def dit_attn_gemm_fp8(a, w, a_scale: float, w_scale: float, y=None, *, stream=No
         y = torch.empty(tuple(a.shape[:-1]) + (N,), dtype=torch.bfloat16, device=a.device)
     _require(y, "y", (torch.bfloat16,), M * N)
     dev = _one_device(a, w, y)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(dit_attn_gemm_fp8_ptr(a.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, float(a_scale),
                                      float(w_scale), _stream_handle(stream, dev)), "dit_attn_gemm_fp8")
     return y
@@ -583,7 +608,7 @@ def dit_attn_mxfp4_tile_scales(scales, K: int, tiled=None, *, stream=None):
     if tiled.numel() < nbytes:
         raise ValueError(f"tiled must hold {nbytes} bytes")
     dev = _one_device(scales, tiled)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(lib().dit_attn_mxfp4_tile_scales(scales.data_ptr(), tiled.data_ptr(), rows, K,
                                                 _stream_handle(stream, dev)), "dit_attn_mxfp4_tile_scales")
     return tiled
@@ -613,7 +638,7 @@ def dit_attn_gemm_mxfp4(a, a_scales_tiled, w, w_scales_tiled, y=None, *, stream=
         y = torch.empty(tuple(a.shape[:-1]) + (N,), dtype=torch.bfloat16, device=a.device)
     _require(y, "y", (torch.bfloat16,), M * N)
     dev = _one_device(a, w, a_scales_tiled, w_scales_tiled, y)
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(dit_attn_gemm_mxfp4_ptr(a.data_ptr(), a_scales_tiled.data_ptr(), w.data_ptr(),
                                        w_scales_tiled.data_ptr(), y.data_ptr(), M, N, K,
                                        _stream_handle(stream, dev)), "dit_attn_gemm_mxfp4")
