@@ -425,7 +425,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
 // The kernel (gemm_mxf4_pair_kernel, below) runs on CTA pairs.  Per K stage of
 // 256 elements each CTA loads its share of A and W and their scale atoms,
 // the leader copies the scales into a TMEM ring slot and issues four MMAs of
-// K = 64.  The epilogue reads the whole fp32 accumulator into registers as
+// K = 64.  When every pair can keep one N tile for the whole launch and K is
+// at most 3328, W's scales for all of K are copied into TMEM once per launch
+// and only A's are copied per stage (a third of the copies).  The epilogue reads the whole fp32 accumulator into registers as
 // bf16 and hands TMEM back before it stages and stores the tile, so the next
 // tile's MMAs start while the stores drain.
 
@@ -474,11 +476,23 @@ constexpr int kP4StageB = (kF4BN / 2) * kBKB;     // 16 KB: this CTA's 128 rows 
 constexpr int kP4StageSFA = 1024, kP4StageSFB = 2048;
 constexpr int kP4StageBytes = kP4StageA + kP4StageB + kP4StageSFA + kP4StageSFB;
 
+// Resident W scales.  When each pair works on one 256-column tile of W for
+// the whole launch (n_tiles <= pairs) and K is short enough, the W scale
+// atoms for all of K are loaded once (one 2 KB block per K stage, as the
+// per-stage path lays them out) and copied into TMEM once; each stage then
+// copies only A's scales.  TMEM: accumulator 0..255, A scale ring
+// 256 + 8 s, W scales from kF4ResSfb at 16 per K stage.
+constexpr uint32_t kF4ResSfa = kF4TmemSf;                           // A scale slot s at + 8 s
+constexpr uint32_t kF4ResSfb = kF4ResSfa + 8 * kP4Stages;          // 296: W scales of stage k at + 16 k
+constexpr int kF4ResMaxStages = (int)(kTmemCols - kF4ResSfb) / 16; // 13: K <= 3328
+constexpr int kP4StageBytesRes = kP4StageA + kP4StageB + kP4StageSFA;
+
 struct P4Bars {
     uint64_t full[kP4Stages];   // leader: stage s of both CTAs landed
     uint64_t empty[kP4Stages];  // each CTA: the MMAs reading stage s completed
     uint64_t tfull;             // each CTA: the accumulator holds a finished tile
     uint64_t tempty;            // leader: both CTAs' epilogues have read it
+    uint64_t sfb_full;          // leader: both CTAs' resident W scale atoms landed
     uint64_t drain;
     uint32_t tmem_base;
     uint32_t abort;
@@ -490,11 +504,39 @@ struct P4Smem {
     static constexpr int OFF_SFA = OFF_B + kP4Stages * kP4StageB;
     static constexpr int OFF_SFB = OFF_SFA + kP4Stages * kP4StageSFA;
     static constexpr int OFF_O = OFF_SFB + kP4Stages * kP4StageSFB;
-    static constexpr int OFF_BAR = OFF_O + kOStage;
+    static constexpr int OFF_SFB_ALL = OFF_O + kOStage;            // resident W scales
+    static constexpr int OFF_BAR = OFF_SFB_ALL + kF4ResMaxStages * kP4StageSFB;
     static constexpr int BYTES = OFF_BAR + 256 + 1024;
 };
 static_assert(P4Smem::BYTES <= 232448, "shared memory budget");
 static_assert(kF4TmemSf + kP4Stages * kF4SfCols <= kTmemCols, "TMEM budget");
+static_assert(kF4ResSfb + 16 * kF4ResMaxStages <= kTmemCols, "TMEM budget (resident W scales)");
+
+// The k-th tile of this pair (false when it has no more).  Per-stage scales:
+// tiles t = pair + k * pairs, the 12-ish N tiles of one A block consecutive.
+// Resident W scales: pair p keeps N tile p % n_tiles, and the pairs sharing it
+// take every c-th 256-row block of A.
+template <bool RES>
+__device__ __forceinline__ bool p4_tile(const F4Params &p, int k, int &m0, int &n0)
+{
+    const int pair = (int)blockIdx.x / 2, pairs = (int)gridDim.x / 2;
+    if (RES) {
+        const int n = pair % p.n_tiles, i = pair / p.n_tiles;
+        const int c = pairs / p.n_tiles + (n < pairs % p.n_tiles ? 1 : 0);
+        const long long m = i + (long long)k * c;
+        if (m >= p.m_tiles)
+            return false;
+        m0 = (int)m * 2 * kF4BM;
+        n0 = n * kF4BN;
+        return true;
+    }
+    const long long t = pair + (long long)k * pairs;
+    if (t >= (long long)p.m_tiles * p.n_tiles)
+        return false;
+    m0 = (int)(t / p.n_tiles) * 2 * kF4BM;
+    n0 = (int)(t % p.n_tiles) * kF4BN;
+    return true;
+}
 
 __device__ __forceinline__ void mma2_mxf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
                                           uint32_t sfb, uint32_t acc)
@@ -520,6 +562,7 @@ struct P4Ctx {
     __device__ uint32_t leader_bar(const uint64_t &b) const { return mapa_shared(smem_u32(&b), 0); }
 };
 
+template <bool RES>
 __device__ __forceinline__ void p4_producer(const P4Ctx &x, const F4Params &p, const CUtensorMap *tm_a,
                                             const CUtensorMap *tm_w, const CUtensorMap *tm_sa,
                                             const CUtensorMap *tm_sw)
@@ -527,10 +570,19 @@ __device__ __forceinline__ void p4_producer(const P4Ctx &x, const F4Params &p, c
     const uint64_t pol_a = l2_policy_evict_last();
     const uint64_t pol_w = l2_policy_evict_last();
     const bool leader = x.rank == 0;
-    const int tiles = p.m_tiles * p.n_tiles;
+    int m0 = 0, n0 = 0;
+    if (RES && p4_tile<RES>(p, 0, m0, n0)) {
+        // This pair's W scale atoms for all of K, once (the N tile never changes).
+        const uint32_t sfb_full = x.leader_bar(x.bars->sfb_full);
+        if (leader)
+            mbar_arrive_expect_tx(x.bar(x.bars->sfb_full), 2 * p.kb * kP4StageSFB);
+        for (int k = 0; k < p.kb; ++k)
+            for (int b = 0; b < 2; ++b)
+                tma_load_2d_pair(x.base + P4Smem::OFF_SFB_ALL + k * kP4StageSFB + b * 1024, tm_sw, sfb_full, 0,
+                                 ((n0 / 128 + b) * p.groups + 2 * k) * 2, pol_w);
+    }
     int it = 0;
-    for (int t = blockIdx.x / 2; t < tiles; t += gridDim.x / 2) {
-        const int m0 = (t / p.n_tiles) * 2 * kF4BM, n0 = (t % p.n_tiles) * kF4BN;
+    for (int tk = 0; p4_tile<RES>(p, tk, m0, n0); ++tk) {
         const int rba = m0 / 128 + (int)x.rank, rbw = n0 / 128;
         for (int k = 0; k < p.kb; ++k, ++it) {
             const int s = it % kP4Stages;
@@ -538,7 +590,7 @@ __device__ __forceinline__ void p4_producer(const P4Ctx &x, const F4Params &p, c
                 !wait_bar(x.bar(x.bars->empty[s]), ((it / kP4Stages) - 1) & 1, x.abort, x.lim, kSiteEmpty))
                 return;
             if (leader)
-                mbar_arrive_expect_tx(x.bar(x.bars->full[s]), 2 * kP4StageBytes);
+                mbar_arrive_expect_tx(x.bar(x.bars->full[s]), 2 * (RES ? kP4StageBytesRes : kP4StageBytes));
             const uint32_t full = x.leader_bar(x.bars->full[s]);
             tma_load_2d_pair(x.base + P4Smem::OFF_A + s * kP4StageA, tm_a, full, k * kBKB, m0 + (int)x.rank * kF4BM,
                              pol_a);
@@ -547,13 +599,15 @@ __device__ __forceinline__ void p4_producer(const P4Ctx &x, const F4Params &p, c
             // scale atoms of groups 2k, 2k+1: 4 rows of 256 bytes from (block * G + 2k) * 2
             tma_load_2d_pair(x.base + P4Smem::OFF_SFA + s * kP4StageSFA, tm_sa, full, 0, (rba * p.groups + 2 * k) * 2,
                              pol_a);
-            for (int b = 0; b < 2; ++b)
-                tma_load_2d_pair(x.base + P4Smem::OFF_SFB + s * kP4StageSFB + b * 1024, tm_sw, full, 0,
-                                 ((rbw + b) * p.groups + 2 * k) * 2, pol_w);
+            if (!RES)
+                for (int b = 0; b < 2; ++b)
+                    tma_load_2d_pair(x.base + P4Smem::OFF_SFB + s * kP4StageSFB + b * 1024, tm_sw, full, 0,
+                                     ((rbw + b) * p.groups + 2 * k) * 2, pol_w);
         }
     }
 }
 
+template <bool RES>
 __device__ __forceinline__ void p4_mma(const P4Ctx &x, const F4Params &p)
 {
     constexpr uint16_t kBoth = 0x3;
@@ -563,10 +617,26 @@ __device__ __forceinline__ void p4_mma(const P4Ctx &x, const F4Params &p)
     const uint64_t b_desc = make_smem_desc(base + P4Smem::OFF_B, 16, 8 * 128, kSwizzle128B);
     const uint64_t sfa_desc = make_smem_desc(base + P4Smem::OFF_SFA, 2048, 128, kSwizzleNone);
     const uint64_t sfb_desc = make_smem_desc(base + P4Smem::OFF_SFB, 2048, 128, kSwizzleNone);
-    const int tiles = p.m_tiles * p.n_tiles;
     bool ok = true;
-    int it = 0, local = 0;
-    for (int t = blockIdx.x / 2; t < tiles && ok; t += gridDim.x / 2, ++local) {
+    int it = 0, local = 0, m0 = 0, n0 = 0;
+    if (RES && p4_tile<RES>(p, 0, m0, n0)) {
+        // The resident W scales: stage k's 2 KB block (groups 2k, 2k+1; row blocks
+        // 0, 1) into columns kF4ResSfb + 16 k + 8 g + 4 b, as the per-stage path does.
+        const uint64_t all_desc = make_smem_desc(base + P4Smem::OFF_SFB_ALL, 2048, 128, kSwizzleNone);
+        ok = __all_sync(0xffffffffu, wait_bar(x.bar(x.bars->sfb_full), 0, x.abort, x.lim, kSiteFull));
+        if (ok) {
+            tc_fence_after();
+            if (elect_one()) {
+                for (int k = 0; k < p.kb; ++k)
+                    for (int g = 0; g < 2; ++g)
+                        for (int b = 0; b < 2; ++b)
+                            tmem_cp2_32x128_x4(tmem + kF4ResSfb + 16 * k + 8 * g + 4 * b,
+                                               all_desc + ((uint32_t)(k * kP4StageSFB + b * 1024 + g * 512) >> 4));
+            }
+            __syncwarp();
+        }
+    }
+    for (int tk = 0; ok && p4_tile<RES>(p, tk, m0, n0); ++tk, ++local) {
         if (local >= 1)
             ok = __all_sync(0xffffffffu,
                             wait_bar(x.bar(x.bars->tempty), (local - 1) & 1, x.abort, x.lim, kSiteTmemEmpty));
@@ -575,22 +645,35 @@ __device__ __forceinline__ void p4_mma(const P4Ctx &x, const F4Params &p)
         tc_fence_after();
         for (int k = 0; k < p.kb && ok; ++k, ++it) {
             const int s = it % kP4Stages;
-            ok = __all_sync(0xffffffffu,
-                            wait_bar(x.bar(x.bars->full[s]), (it / kP4Stages) & 1, x.abort, x.lim, kSiteFull));
-            if (!ok)
-                break;
-            tc_fence_after();
-            const uint32_t sfa_t = tmem + kF4TmemSf + (uint32_t)s * kF4SfCols;
-            const uint32_t sfb_t = sfa_t + 8;
-            if (elect_one()) {
-                for (int g = 0; g < 2; ++g) {
-                    tmem_cp2_32x128_x4(sfa_t + 4 * g, sfa_desc + ((uint32_t)(s * kP4StageSFA + g * 512) >> 4));
-                    for (int b = 0; b < 2; ++b)
-                        tmem_cp2_32x128_x4(sfb_t + 8 * g + 4 * b,
-                                           sfb_desc + ((uint32_t)(s * kP4StageSFB + b * 1024 + g * 512) >> 4));
+            const uint32_t sfa_t = RES ? tmem + kF4ResSfa + 8u * (uint32_t)s : tmem + kF4TmemSf + (uint32_t)s * kF4SfCols;
+            const uint32_t sfb_t = RES ? tmem + kF4ResSfb + 16u * (uint32_t)k : sfa_t + 8;
+            // A run of scale copies between MMAs costs about the same whatever its
+            // length, so with resident W scales the A scales of two K stages are
+            // copied together (at even k, once both stages have landed).
+            if (!RES || (k & 1) == 0) {
+                const bool pair_k = RES && k + 1 < p.kb;
+                const int s2 = (it + 1) % kP4Stages;
+                ok = __all_sync(0xffffffffu,
+                                wait_bar(x.bar(x.bars->full[s]), (it / kP4Stages) & 1, x.abort, x.lim, kSiteFull) &&
+                                    (!pair_k || wait_bar(x.bar(x.bars->full[s2]), ((it + 1) / kP4Stages) & 1,
+                                                         x.abort, x.lim, kSiteFull)));
+                if (!ok)
+                    break;
+                tc_fence_after();
+                if (elect_one()) {
+                    for (int g = 0; g < 2; ++g) {
+                        tmem_cp2_32x128_x4(sfa_t + 4 * g, sfa_desc + ((uint32_t)(s * kP4StageSFA + g * 512) >> 4));
+                        if (pair_k)
+                            tmem_cp2_32x128_x4(tmem + kF4ResSfa + 8u * (uint32_t)s2 + 4 * g,
+                                               sfa_desc + ((uint32_t)(s2 * kP4StageSFA + g * 512) >> 4));
+                        if (!RES)
+                            for (int b = 0; b < 2; ++b)
+                                tmem_cp2_32x128_x4(sfb_t + 8 * g + 4 * b,
+                                                   sfb_desc + ((uint32_t)(s * kP4StageSFB + b * 1024 + g * 512) >> 4));
+                    }
                 }
+                __syncwarp();
             }
-            __syncwarp();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const int g = kk >> 1;
@@ -618,6 +701,7 @@ __device__ __forceinline__ void p4_mma(const P4Ctx &x, const F4Params &p)
     }
 }
 
+template <bool RES>
 __device__ __forceinline__ void p4_epilogue(const P4Ctx &x, const F4Params &p, const CUtensorMap *tm_y, int warp,
                                             int lane)
 {
@@ -625,12 +709,11 @@ __device__ __forceinline__ void p4_epilogue(const P4Ctx &x, const F4Params &p, c
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const bool issuer = warp == kEpiWarp0 && lane == 0;
-    const int tiles = p.m_tiles * p.n_tiles;
     const uint32_t tempty_leader = x.leader_bar(x.bars->tempty);
     bool ok = true;
-    int local = 0;
-    for (int t = blockIdx.x / 2; t < tiles && ok; t += gridDim.x / 2, ++local) {
-        const int m0 = (t / p.n_tiles) * 2 * kF4BM + (int)x.rank * kF4BM, n0 = (t % p.n_tiles) * kF4BN;
+    int local = 0, mp = 0, n0 = 0;
+    for (int tk = 0; ok && p4_tile<RES>(p, tk, mp, n0); ++tk, ++local) {
+        const int m0 = mp + (int)x.rank * kF4BM;
         ok = __all_sync(0xffffffffu, wait_bar(x.bar(x.bars->tfull), local & 1, x.abort, x.lim, kSiteTmemFull));
         if (!bar_and(1, 128, ok)) {
             ok = false;
@@ -681,6 +764,7 @@ __device__ __forceinline__ void p4_epilogue(const P4Ctx &x, const F4Params &p, c
         bulk_wait_group_all();
 }
 
+template <bool RES>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
                       const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_sa,
@@ -700,6 +784,7 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_con
         }
         mbar_init(smem_u32(&bars->tfull), 1);
         mbar_init(smem_u32(&bars->tempty), 8);           // 4 epilogue warps x 2 CTAs
+        mbar_init(smem_u32(&bars->sfb_full), 1);
         mbar_init(smem_u32(&bars->drain), 1);
         bars->abort = 0u;
         fence_barrier_init();
@@ -730,12 +815,12 @@ gemm_mxf4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_con
 
     if (warp == 0) {
         if (lane == 0)
-            p4_producer(x, p, &tm_a, &tm_w, &tm_sa, &tm_sw);
+            p4_producer<RES>(x, p, &tm_a, &tm_w, &tm_sa, &tm_sw);
     } else if (warp == 1) {
         if (rank == 0)
-            p4_mma(x, p);
+            p4_mma<RES>(x, p);
     } else {
-        p4_epilogue(x, p, &tm_y, warp, lane);
+        p4_epilogue<RES>(x, p, &tm_y, warp, lane);
     }
 
     tc_fence_before();

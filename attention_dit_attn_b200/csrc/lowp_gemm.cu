@@ -192,10 +192,11 @@ int dit_attn_gemm_mxfp4(const void *a, const void *a_scales, const void *w, cons
         return rc;
     if (!dit_abi::device_buffers(device, {a, w, y, a_scales, w_scales}))
         return DIT_ATTN_ERR_DEVICE;
-    auto kern = dit_gemm::gemm_mxf4_pair_kernel;
     if (g_attr_set_f4[device].load(std::memory_order_acquire) == 0) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dit_gemm::P4Smem::BYTES) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(dit_gemm::gemm_mxf4_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dit_gemm::P4Smem::BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(dit_gemm::gemm_mxf4_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dit_gemm::P4Smem::BYTES) != cudaSuccess)
             return DIT_ATTN_ERR_LAUNCH;
         g_attr_set_f4[device].store(1, std::memory_order_release);
     }
@@ -231,6 +232,9 @@ int dit_attn_gemm_mxfp4(const void *a, const void *a_scales, const void *w, cons
         return DIT_ATTN_ERR_LAUNCH;
     const long long tiles = (long long)p.m_tiles * p.n_tiles;
     const long long clusters = tiles < sms / 2 ? tiles : sms / 2;
+    // W scales resident in TMEM when every pair keeps one N tile and K fits.
+    const bool resident = p.n_tiles <= clusters && p.kb <= dit_gemm::kF4ResMaxStages;
+    auto kern = resident ? dit_gemm::gemm_mxf4_pair_kernel<true> : dit_gemm::gemm_mxf4_pair_kernel<false>;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * clusters));
     cfg.blockDim = dim3(dit_gemm::kThreads);

@@ -80,6 +80,9 @@ def test_tile_scales_is_the_layout(cuda_lib, rows, K):
     (300, 264, 512),       # two N tiles, the second with a single scale block
     (1000, 768, 1024),     # several tiles in M and N
     (128, 256, 3072),      # one tile, a long K
+    (256, 256, 3584),      # K past what TMEM holds of W's scales: per-stage W scales
+    (300, 19200, 64),      # more N tiles than CTA pairs: per-stage W scales
+    (1100, 264, 3328),     # the longest K with resident W scales, pairs sharing an N tile
 ])
 def test_gemm_mxfp4_matches_the_oracle(cuda_lib, M, N, K):
     a, sa, w, sw = wl.gemm_operands_mxfp4(M, N, K, seed=M + N + K)
