@@ -425,9 +425,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
 // The kernel (gemm_mxf4_pair_kernel, below) runs on CTA pairs.  Per K stage of
 // 256 elements each CTA loads its share of A and W and their scale atoms,
 // the leader copies the scales into a TMEM ring slot and issues four MMAs of
-// K = 64.  When every pair can keep one N tile for the whole launch and K is
-// at most 3328, W's scales for all of K are copied into TMEM once per launch
-// and only A's are copied per stage (a third of the copies).  The epilogue reads the whole fp32 accumulator into registers as
+// K = 64.  When every pair can keep one N tile for the whole launch, K is at
+// most 3328 and A fits in L2 (the host's choice), W's scales for all of K are
+// copied into TMEM once per launch and only A's are copied per stage, two
+// stages per run of copies.  The epilogue reads the whole fp32 accumulator into registers as
 // bf16 and hands TMEM back before it stages and stores the tile, so the next
 // tile's MMAs start while the stores drain.
 

@@ -232,8 +232,12 @@ int dit_attn_gemm_mxfp4(const void *a, const void *a_scales, const void *w, cons
         return DIT_ATTN_ERR_LAUNCH;
     const long long tiles = (long long)p.m_tiles * p.n_tiles;
     const long long clusters = tiles < sms / 2 ? tiles : sms / 2;
-    // W scales resident in TMEM when every pair keeps one N tile and K fits.
-    const bool resident = p.n_tiles <= clusters && p.kb <= dit_gemm::kF4ResMaxStages;
+    // W scales resident in TMEM when every pair keeps one N tile and K fits.  That
+    // walk has the pairs of different N tiles reach a block of A at different
+    // times, which only costs nothing while all of A stays in L2 (126 MB): at most
+    // 64 MB of A codes.
+    const bool resident = p.n_tiles <= clusters && p.kb <= dit_gemm::kF4ResMaxStages &&
+                          M * (long long)(K / 2) <= (64ll << 20);
     auto kern = resident ? dit_gemm::gemm_mxf4_pair_kernel<true> : dit_gemm::gemm_mxf4_pair_kernel<false>;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * clusters));

@@ -135,3 +135,15 @@ def test_gemm_mxfp4_is_deterministic_and_writes_only_y(cuda_lib):
     assert torch.equal(y1.view(torch.int16), y.view(torch.int16))
     assert bool((guard[M * N:] == 7.0).all())
     _check(y.cpu(), a, sa, w, sw)
+
+
+def test_gemm_mxfp4_large_activation_takes_the_per_stage_path_sampled_rows(cuda_lib):
+    """Four times the projection's tokens (M = 135168, 208 MB of codes, more than
+    the 64 MB for which W's scales are kept in TMEM): the per-stage scale path on
+    a full-size launch; the oracle checks 64 sampled rows."""
+    M, N, K = 4 * wl.GEMM_SHAPES["flux_2048_cfg_proj"][0], 3072, 3072
+    a, sa, w, sw = wl.gemm_operands_mxfp4(M, N, K, seed=8)
+    y = _gemm_gpu(a, sa, w, sw, K)
+    rows = np.sort(np.random.default_rng(9).choice(M, 64, replace=False))
+    rows[0], rows[-1] = 0, M - 1
+    _check(y, a, sa, w, sw, rows)
