@@ -136,6 +136,16 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     }
 }
 
+// Abort path of a producer (a wait ran out of time): give the tile loads it
+// already issued 1 ms to land before the CTA leaves, far above a tile load's
+// latency, so none writes into shared memory the SM has handed on.
+__device__ __forceinline__ void pause_for_loads_in_flight()
+{
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 1000000ull) {
+    }
+}
+
 __device__ __forceinline__ void named_bar(uint32_t id, uint32_t n)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -198,8 +208,10 @@ __device__ __forceinline__ void producer(const Ctx &x, const GemmParams &p, cons
         for (int k = 0; k < p.kb; ++k, ++it) {
             const int s = it % kStages;
             if (it >= kStages &&
-                !wait_bar(x.bar(x.bars->empty[s]), ((it / kStages) - 1) & 1, x.abort, x.lim, kSiteEmpty))
+                !wait_bar(x.bar(x.bars->empty[s]), ((it / kStages) - 1) & 1, x.abort, x.lim, kSiteEmpty)) {
+                pause_for_loads_in_flight();
                 return;
+            }
             if (leader)
                 mbar_arrive_expect_tx(x.bar(x.bars->full[s]), 2 * (kStageA + kStageB));
             const uint32_t full = x.leader_bar(x.bars->full[s]);
@@ -588,8 +600,10 @@ __device__ __forceinline__ void p4_producer(const P4Ctx &x, const F4Params &p, c
         for (int k = 0; k < p.kb; ++k, ++it) {
             const int s = it % kP4Stages;
             if (it >= kP4Stages &&
-                !wait_bar(x.bar(x.bars->empty[s]), ((it / kP4Stages) - 1) & 1, x.abort, x.lim, kSiteEmpty))
+                !wait_bar(x.bar(x.bars->empty[s]), ((it / kP4Stages) - 1) & 1, x.abort, x.lim, kSiteEmpty)) {
+                pause_for_loads_in_flight();
                 return;
+            }
             if (leader)
                 mbar_arrive_expect_tx(x.bar(x.bars->full[s]), 2 * (RES ? kP4StageBytesRes : kP4StageBytes));
             const uint32_t full = x.leader_bar(x.bars->full[s]);
