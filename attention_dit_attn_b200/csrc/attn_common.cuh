@@ -25,7 +25,15 @@ constexpr int kBM = 128;             // query rows per tile (MMA M)
 constexpr int kBN = 128;             // keys per K/V tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleLog2 = 8.0f; // lazy-rescale threshold (p <= 256)
+// Lazy rescaling.  bf16 path: each tile's max is taken, and the running max
+// is raised only when a tile's exceeds it by more than kRescaleLog2 (p <= 256).
+// FP8 path, without a per-tile max: a half-row keeps the running max of its
+// first key tile, so a later tile's p = 2^(x - m) may exceed 1.  The sum of
+// the thread's p over a tile bounds each of them; when that sum reaches
+// kPGuardF16 (or is not finite) the warp takes the rescale path: the tile's
+// max, O and l scaled down, P recomputed.  f16 P must stay below 65504.
+constexpr float kRescaleLog2 = 8.0f;
+constexpr float kPGuardF16 = 32768.0f;                   // 2^15
 
 // bf16 P is the high half of the f32 p (one byte permute, i.e. truncation).
 // That drops 16 mantissa bits: on average over the dropped bits the loss is
@@ -156,15 +164,24 @@ __device__ __forceinline__ float max3f(float a, float b, float c)
 // f in [-1/2, 1/2]; 2^f is a cubic fitted for minimum max relative error on
 // [-1/2, 1/2] (max rel. error 7.5e-5, below the half-ulp of bf16 and f16 P);
 // 2^n is added to the exponent field.  x is clamped to >= -126 so the
-// exponent never underflows; the callers guarantee x <= 9.
+// exponent never underflows.  With CLAMP_HI (FP8 path, whose x is not bounded
+// by a per-tile max) x is also clamped to <= 127, so the exponent field never
+// wraps: a larger x gives 2^127, which the caller's guard on the sum of p
+// catches as it catches MUFU's +inf; the bf16 path guarantees x <= 9.
 constexpr float kPolyC0 = 0.9999281167984009f, kPolyC1 = 0.6932609677314758f,
                 kPolyC2 = 0.24261052906513214f, kPolyC3 = 0.05517127364873886f;
 constexpr float kRintMagic = 12582912.0f;   // 1.5 * 2^23
 
+template <bool CLAMP_HI = false>
 __device__ __forceinline__ float2 exp2_poly2(float2 x)
 {
-    x.x = fmaxf(x.x, -126.f);
-    x.y = fmaxf(x.y, -126.f);
+    if (CLAMP_HI) {
+        x.x = fminf(fmaxf(x.x, -126.f), 127.f);
+        x.y = fminf(fmaxf(x.y, -126.f), 127.f);
+    } else {
+        x.x = fmaxf(x.x, -126.f);
+        x.y = fmaxf(x.y, -126.f);
+    }
     const float2 t = __fadd2_rn(x, make_float2(kRintMagic, kRintMagic));
     const float2 n = __fadd2_rn(t, make_float2(-kRintMagic, -kRintMagic));
     const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);

@@ -427,7 +427,7 @@ __device__ __forceinline__ float half_row_exp_store(const uint32_t (&s)[2][32], 
                                          c2c2, nmc);
             float2 e;
             if ((pi & 7) >= 8 - EMU) {
-                e = exp2_poly2(xv);
+                e = exp2_poly2<C::FP8>(xv);
             } else {
                 e.x = ex2_approx(xv.x);
                 e.y = ex2_approx(xv.y);
@@ -476,18 +476,53 @@ __device__ __forceinline__ void half_row_step(const PairCtx<C> &x, const FwdPara
     tmem_wait_ld_regs(s[0]);
     tmem_wait_ld_regs(s[1]);
     const bool masked = j == n - 1 && p.kv_tail < kBN;
-    const float mx = masked ? half_row_max<true>(s, 64 * h, p.kv_tail) : half_row_max<false>(s, 64 * h, kBN);
-    float alpha = 1.f;
-    if (j == 0) {
-        st.m_use = mx;
-    } else if ((mx - st.m_use) * st.c2 > kRescaleLog2) {
-        alpha = ex2_approx((st.m_use - mx) * st.c2);
-        st.m_use = mx;
-    }
+    auto tile_max = [&]() {
+        return masked ? half_row_max<true>(s, 64 * h, p.kv_tail) : half_row_max<false>(s, 64 * h, kBN);
+    };
     // bf16 P is truncated; kTruncLog2 makes it unbiased (attn_common.cuh).
-    const float mc = st.m_use * st.c2 - (C::FP8 ? 0.f : kTruncLog2);
-    const float sum = masked ? half_row_exp_store<C, true, C::EXP_EMU>(s, tS, 64 * h, p.kv_tail, st.c2, mc)
-                             : half_row_exp_store<C, false, C::EXP_EMU>(s, tS, 64 * h, kBN, st.c2, mc);
+    auto exp_store = [&]() {
+        const float mc = st.m_use * st.c2 - (C::FP8 ? 0.f : kTruncLog2);
+        return masked ? half_row_exp_store<C, true, C::EXP_EMU>(s, tS, 64 * h, p.kv_tail, st.c2, mc)
+                      : half_row_exp_store<C, false, C::EXP_EMU>(s, tS, 64 * h, kBN, st.c2, mc);
+    };
+    float alpha = 1.f;
+    float sum;
+    if constexpr (C::FP8) {
+        // FP8 path (f16 P, rounded to nearest): the first tile sets the running
+        // max; later tiles use it as it stands, and only the guard on their sum
+        // of p sends a warp back through the max (attn_common.cuh).  tcgen05.st
+        // is warp-wide, so the whole warp recomputes and stores P; lanes whose
+        // max did not move store the same values again.
+        if (j == 0)
+            st.m_use = tile_max();
+        sum = exp_store();
+        if (j > 0) {
+            const bool over = !(sum < kPGuardF16);
+            if (__any_sync(0xffffffffu, over)) {
+                if (over) {
+                    const float mx = tile_max();
+                    if (mx > st.m_use) {
+                        alpha = ex2_approx((st.m_use - mx) * st.c2);
+                        st.m_use = mx;
+                    }
+                }
+                sum = exp_store();
+            }
+        }
+    } else {
+        // bf16 path (P truncated to 8 significant bits): the max of every tile,
+        // raised lazily once it exceeds the running max by kRescaleLog2, so p
+        // stays near 1 for the rows a few keys dominate, where P's truncation
+        // sets the error.
+        const float mx = tile_max();
+        if (j == 0) {
+            st.m_use = mx;
+        } else if ((mx - st.m_use) * st.c2 > kRescaleLog2) {
+            alpha = ex2_approx((st.m_use - mx) * st.c2);
+            st.m_use = mx;
+        }
+        sum = exp_store();
+    }
     st.l = st.l * alpha + sum;
     if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // Rescale this thread's row of O_h once PV(j-1) has finished with it.

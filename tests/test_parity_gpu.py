@@ -54,6 +54,40 @@ def test_peaked_rows_with_lazy_rescale(cuda_lib):
     parity.check(parity.compare(o, lse, o_ref, lse_ref), "bf16")
 
 
+def _jump_inputs(D: int, dtype: str, seed: int):
+    """Rows whose running max jumps by far more than the lazy-rescale guard in
+    later key tiles.  Every query has q[..., 0] = 8 (one head) or 2 (the other);
+    key 300 (third tile) and key 650 (sixth tile) get k[..., 0] = 80 and 150, so
+    their logits exceed the first tile's by tens to hundreds of log2 units: past
+    the bf16 guard (2^64), past MUFU's and the cubic's range (2^128), and far
+    past the f16 guard (2^15)."""
+    g = torch.Generator().manual_seed(seed)
+    B, H, L = 1, 2, 700
+    q = torch.randn((B, H, L, D), generator=g) * 0.5
+    k = torch.randn((B, H, L, D), generator=g) * 0.5
+    v = torch.randn((B, H, L, D), generator=g)
+    q[:, 0, :, 0] = 8.0
+    q[:, 1, :, 0] = 2.0
+    k[:, :, 300, 0] = 80.0
+    k[:, :, 650, 0] = 150.0
+    if dtype == "bf16":
+        return wl.Inputs(q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16), None, None, None)
+    (qq, qs), (kq, ks), (vq, vs) = (wl.quantize_e4m3_per_head(t) for t in (q, k, v))
+    return wl.Inputs(qq, kq, vq, qs, ks, vs)
+
+
+@pytest.mark.parametrize("D,dtype", [(128, "bf16"), (64, "bf16"), (64, "e4m3"), (128, "e4m3")])
+def test_max_jumps_past_the_lazy_rescale_guard(cuda_lib, D, dtype):
+    """The running max of a row is kept from its first key tile; later tiles are
+    only checked through the sum of their p.  Jumps of tens to hundreds of log2
+    units in later tiles must take the rescale path and still match the oracle."""
+    inp = _jump_inputs(D, dtype, seed=40 + D)
+    o, lse = parity.run_gpu(inp, 1 / math.sqrt(D))
+    assert torch.isfinite(o.to(torch.float32)).all() and torch.isfinite(lse).all()
+    o_ref, lse_ref = parity.run_oracle(inp, 1 / math.sqrt(D))
+    parity.check(parity.compare(o, lse, o_ref, lse_ref), dtype)
+
+
 def test_scale_zero_gives_mean_of_v(cuda_lib):
     inp = wl.generate(1, 2, 300, 128, "bf16", seed=12)
     o, lse = parity.run_gpu(inp, 0.0)
