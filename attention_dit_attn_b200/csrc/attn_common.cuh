@@ -25,27 +25,15 @@ constexpr int kBM = 128;             // query rows per tile (MMA M)
 constexpr int kBN = 128;             // keys per K/V tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-// Lazy rescaling.  bf16 path: each tile's max is taken, and the running max
-// is raised only when a tile's exceeds it by more than kRescaleLog2 (p <= 256).
-// FP8 path, without a per-tile max: a half-row keeps the running max of its
-// first key tile, so a later tile's p = 2^(x - m) may exceed 1.  The sum of
-// the thread's p over a tile bounds each of them; when that sum reaches
-// kPGuardF16 (or is not finite) the warp takes the rescale path: the tile's
-// max, O and l scaled down, P recomputed.  f16 P must stay below 65504.
-constexpr float kRescaleLog2 = 8.0f;
+// Lazy rescaling without a per-tile max: a half-row keeps the running max of
+// its first key tile, so a later tile's p = 2^(x - m) may exceed 1.  The sum
+// of the thread's p over a tile bounds each of them; when that sum reaches the
+// guard (or is not finite) the warp takes the rescale path: the tile's max,
+// O and l scaled down, P recomputed.  f16 P (FP8 path) must stay below 65504;
+// bf16 P and the fp32 accumulators (O, l) have room for 2^64 per p.
 constexpr float kPGuardF16 = 32768.0f;                   // 2^15
+constexpr float kPGuardBF16 = 18446744073709551616.0f;   // 2^64
 
-// bf16 P is the high half of the f32 p (one byte permute, i.e. truncation).
-// That drops 16 mantissa bits: on average over the dropped bits the loss is
-// 2^-8 / (1+m) of p, where 1+m is p's significand.  For p = 2^x with x spread
-// over many units, 1+m is log-uniform on [1, 2), where E[1/(1+m)] =
-// 1/(2 ln 2), so the mean relative loss is mu = 1/(512 ln 2) = 2.818e-3.
-// Every p is computed as p * kTruncGain, kTruncGain = 1/(1 - mu) (an offset
-// of kTruncLog2 on the exponent), which makes the truncated value unbiased;
-// the running sums then carry the same factor, which the epilogue takes out of
-// O and the LSE.
-constexpr float kTruncGain = 1.0028257f;
-constexpr float kTruncLog2 = 0.0040709f;   // log2(kTruncGain)
 
 // Wait sites recorded in the error word (bits 8..15).
 enum : uint32_t {
@@ -163,25 +151,18 @@ __device__ __forceinline__ float max3f(float a, float b, float c)
 // n = rint(x) (adding 1.5*2^23 leaves rint(x) in the low mantissa bits) and
 // f in [-1/2, 1/2]; 2^f is a cubic fitted for minimum max relative error on
 // [-1/2, 1/2] (max rel. error 7.5e-5, below the half-ulp of bf16 and f16 P);
-// 2^n is added to the exponent field.  x is clamped to >= -126 so the
-// exponent never underflows.  With CLAMP_HI (FP8 path, whose x is not bounded
-// by a per-tile max) x is also clamped to <= 127, so the exponent field never
-// wraps: a larger x gives 2^127, which the caller's guard on the sum of p
-// catches as it catches MUFU's +inf; the bf16 path guarantees x <= 9.
+// 2^n is added to the exponent field.  x is clamped to [-126, 127], so the
+// exponent field neither underflows nor wraps: a larger x (x is not bounded by
+// a per-tile max) gives 2^127, which the caller's guard on the sum of p
+// catches as it catches MUFU's +inf.
 constexpr float kPolyC0 = 0.9999281167984009f, kPolyC1 = 0.6932609677314758f,
                 kPolyC2 = 0.24261052906513214f, kPolyC3 = 0.05517127364873886f;
 constexpr float kRintMagic = 12582912.0f;   // 1.5 * 2^23
 
-template <bool CLAMP_HI = false>
 __device__ __forceinline__ float2 exp2_poly2(float2 x)
 {
-    if (CLAMP_HI) {
-        x.x = fminf(fmaxf(x.x, -126.f), 127.f);
-        x.y = fminf(fmaxf(x.y, -126.f), 127.f);
-    } else {
-        x.x = fmaxf(x.x, -126.f);
-        x.y = fmaxf(x.y, -126.f);
-    }
+    x.x = fminf(fmaxf(x.x, -126.f), 127.f);
+    x.y = fminf(fmaxf(x.y, -126.f), 127.f);
     const float2 t = __fadd2_rn(x, make_float2(kRintMagic, kRintMagic));
     const float2 n = __fadd2_rn(t, make_float2(-kRintMagic, -kRintMagic));
     const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);

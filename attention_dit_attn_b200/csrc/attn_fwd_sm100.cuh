@@ -407,8 +407,7 @@ __device__ __forceinline__ float half_row_max(const uint32_t (&s)[2][32], int kb
 // p = 2^(s*c2 - mc) for this thread's 64 values, packed to 16 bits and stored
 // as 32 TMEM columns at tS (over S values only this thread has read).
 // Returns the sum of the p.  Of every 8 pairs, EMU use the FMA-pipe exp2.
-// bf16 P takes the high halves of the two f32 (one byte permute: truncation,
-// made unbiased by the kTruncGain factor the caller folds into mc); f16 P
+// bf16 P (bf16 path) and f16 P (FP8 path) are rounded to nearest even; f16 P
 // (FP8 path) is rounded to nearest.
 template <class C, bool MASK, int EMU>
 __device__ __forceinline__ float half_row_exp_store(const uint32_t (&s)[2][32], uint32_t tS, int kbase, int valid,
@@ -427,7 +426,7 @@ __device__ __forceinline__ float half_row_exp_store(const uint32_t (&s)[2][32], 
                                          c2c2, nmc);
             float2 e;
             if ((pi & 7) >= 8 - EMU) {
-                e = exp2_poly2<C::FP8>(xv);
+                e = exp2_poly2(xv);
             } else {
                 e.x = ex2_approx(xv.x);
                 e.y = ex2_approx(xv.y);
@@ -437,8 +436,7 @@ __device__ __forceinline__ float half_row_exp_store(const uint32_t (&s)[2][32], 
                 e.y = (kbase + 32 * i + c + 1 < valid) ? e.y : 0.f;
             }
             acc[pi & 3] = __fadd2_rn(acc[pi & 3], e);
-            pk[c / 2] = C::FP8 ? pack_p(e.x, e.y, true)
-                               : __byte_perm(__float_as_uint(e.x), __float_as_uint(e.y), 0x7632);
+            pk[c / 2] = pack_p(e.x, e.y, C::FP8);
         }
         tmem_st16(tS + 16 * i, pk);
     }
@@ -479,49 +477,32 @@ __device__ __forceinline__ void half_row_step(const PairCtx<C> &x, const FwdPara
     auto tile_max = [&]() {
         return masked ? half_row_max<true>(s, 64 * h, p.kv_tail) : half_row_max<false>(s, 64 * h, kBN);
     };
-    // bf16 P is truncated; kTruncLog2 makes it unbiased (attn_common.cuh).
     auto exp_store = [&]() {
-        const float mc = st.m_use * st.c2 - (C::FP8 ? 0.f : kTruncLog2);
+        const float mc = st.m_use * st.c2;
         return masked ? half_row_exp_store<C, true, C::EXP_EMU>(s, tS, 64 * h, p.kv_tail, st.c2, mc)
                       : half_row_exp_store<C, false, C::EXP_EMU>(s, tS, 64 * h, kBN, st.c2, mc);
     };
     float alpha = 1.f;
     float sum;
-    if constexpr (C::FP8) {
-        // FP8 path (f16 P, rounded to nearest): the first tile sets the running
-        // max; later tiles use it as it stands, and only the guard on their sum
-        // of p sends a warp back through the max (attn_common.cuh).  tcgen05.st
-        // is warp-wide, so the whole warp recomputes and stores P; lanes whose
-        // max did not move store the same values again.
-        if (j == 0)
-            st.m_use = tile_max();
-        sum = exp_store();
-        if (j > 0) {
-            const bool over = !(sum < kPGuardF16);
-            if (__any_sync(0xffffffffu, over)) {
-                if (over) {
-                    const float mx = tile_max();
-                    if (mx > st.m_use) {
-                        alpha = ex2_approx((st.m_use - mx) * st.c2);
-                        st.m_use = mx;
-                    }
+    // The first tile sets the running max; later tiles use it as it stands, and
+    // only the guard on their sum of p sends a warp back through the max
+    // (attn_common.cuh).  tcgen05.st is warp-wide, so the whole warp recomputes
+    // and stores P; lanes whose max did not move store the same values again.
+    if (j == 0)
+        st.m_use = tile_max();
+    sum = exp_store();
+    if (j > 0) {
+        const bool over = !(sum < (C::FP8 ? kPGuardF16 : kPGuardBF16));
+        if (__any_sync(0xffffffffu, over)) {
+            if (over) {
+                const float mx = tile_max();
+                if (mx > st.m_use) {
+                    alpha = ex2_approx((st.m_use - mx) * st.c2);
+                    st.m_use = mx;
                 }
-                sum = exp_store();
             }
+            sum = exp_store();
         }
-    } else {
-        // bf16 path (P truncated to 8 significant bits): the max of every tile,
-        // raised lazily once it exceeds the running max by kRescaleLog2, so p
-        // stays near 1 for the rows a few keys dominate, where P's truncation
-        // sets the error.
-        const float mx = tile_max();
-        if (j == 0) {
-            st.m_use = mx;
-        } else if ((mx - st.m_use) * st.c2 > kRescaleLog2) {
-            alpha = ex2_approx((st.m_use - mx) * st.c2);
-            st.m_use = mx;
-        }
-        sum = exp_store();
     }
     st.l = st.l * alpha + sum;
     if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -600,7 +581,7 @@ __device__ __forceinline__ void pair_softmax(const PairCtx<C> &x, const FwdParam
     const uint32_t ost = C::FP8 ? x.base + C::OFF_OST : x.base + C::OFF_Q;
     if (alive) {
         tc_fence_after();
-        const float inv = (C::FP8 ? vs : kTruncGain) / l_row;
+        const float inv = (C::FP8 ? vs : 1.f) / l_row;
         const float w0 = a0 * inv, w1 = a1 * inv;
         // This thread writes output columns h*D/2 .. h*D/2 + D/2 of its row.
         const uint32_t tO0 = x.tmem + lane_off + C::TM_O + h * (D / 2);
@@ -632,7 +613,7 @@ __device__ __forceinline__ void pair_softmax(const PairCtx<C> &x, const FwdParam
     if (alive) {
         const int qrow = x.q0 + row;
         if (h == 0 && p.lse != nullptr && qrow < p.L)
-            p.lse[(long long)x.bh * p.L + qrow] = (mrow + log2f(l_row) - (C::FP8 ? 0.f : kTruncLog2)) * kLn2;
+            p.lse[(long long)x.bh * p.L + qrow] = (mrow + log2f(l_row)) * kLn2;
         if (warp == 0 && lane == 0) {
             for (int b = 0; b < C::OBOX; ++b)
                 tma_store_3d(tm_o, ost + b * C::OBOX_BYTES, b * 64, x.q0, x.bh);

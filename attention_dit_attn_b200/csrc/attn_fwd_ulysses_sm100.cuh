@@ -197,7 +197,7 @@ __device__ __forceinline__ void ulysses_softmax(const PairCtx<C> &x, const FwdPa
     const uint32_t ost = C::FP8 ? x.base + C::OFF_OST : x.base + C::OFF_Q;
     if (alive) {
         tc_fence_after();
-        const float inv = (C::FP8 ? vs : kTruncGain) / l_row;
+        const float inv = (C::FP8 ? vs : 1.f) / l_row;
         const float w0 = a0 * inv, w1 = a1 * inv;
         const uint32_t tO0 = x.tmem + lane_off + C::TM_O + h * (D / 2);
 #pragma unroll
@@ -230,7 +230,7 @@ __device__ __forceinline__ void ulysses_softmax(const PairCtx<C> &x, const FwdPa
         if (h == 0 && u.lse[0] != nullptr && qrow < p.L) {
             int c, r;
             shard_of(u, qrow, c, r);
-            u.lse[c][(long long)bhs * u.Ls + r] = (mrow + log2f(l_row) - (C::FP8 ? 0.f : kTruncLog2)) * kLn2;
+            u.lse[c][(long long)bhs * u.Ls + r] = (mrow + log2f(l_row)) * kLn2;
         }
         if (warp == 0 && lane == 0) {
             // Ls and L are multiples of 64: a 64-row half lies in one shard, wholly

@@ -19,8 +19,9 @@ def kernel_coeffs():
 
 
 def exp2_poly_model(x: np.ndarray, c: np.ndarray) -> np.ndarray:
-    """float32 replica of exp2_poly2: clamp, rint via 1.5*2^23, cubic, exponent add."""
-    x = np.maximum(x.astype(np.float32), np.float32(-126.0))
+    """float32 replica of exp2_poly2: clamp to [-126, 127], rint via 1.5*2^23, cubic,
+    exponent add."""
+    x = np.minimum(np.maximum(x.astype(np.float32), np.float32(-126.0)), np.float32(127.0))
     magic = np.float32(12582912.0)
     t = (x + magic).astype(np.float32)
     n = (t - magic).astype(np.float32)
@@ -35,7 +36,8 @@ def test_coefficients_are_the_fit():
 
 
 def test_relative_error_below_bf16_and_f16_half_ulp():
-    x = np.linspace(-60.0, 9.0, 2_000_001, dtype=np.float32)
+    # x above 0 occurs: a later key tile may exceed the running max of the first.
+    x = np.linspace(-60.0, 126.0, 2_000_001, dtype=np.float32)
     got = exp2_poly_model(x, kernel_coeffs()).astype(np.float64)
     rel = np.abs(got / np.exp2(x.astype(np.float64)) - 1)
     assert rel.max() < 1e-4 < 2.0 ** -11     # f16 P half-ulp is 2^-11, bf16 2^-9
@@ -45,3 +47,12 @@ def test_clamped_tail_is_tiny_and_positive():
     x = np.array([-126.0, -200.0, -1e30], dtype=np.float32)
     got = exp2_poly_model(x, kernel_coeffs())
     assert np.all(got >= 0) and np.all(got < 1e-37)
+
+
+def test_clamped_head_is_finite_and_caught_by_the_guard():
+    """x past 127 gives 2^127: finite (no wrap of the exponent field) and far above
+    both guards on the sum of p (2^15 for f16 P, 2^64 for bf16 P)."""
+    x = np.array([127.0, 128.5, 300.0, 1e30], dtype=np.float32)
+    got = exp2_poly_model(x, kernel_coeffs()).astype(np.float64)
+    assert np.all(np.isfinite(got)) and np.all(got > 2.0 ** 126)
+    assert np.all(got >= 2.0 ** 64)
