@@ -42,7 +42,7 @@
 namespace dit {
 
 #ifndef DIT_EXP_EMU
-#define DIT_EXP_EMU 3
+#define DIT_EXP_EMU 2
 #endif
 
 template <int D_, bool FP8_>
