@@ -409,8 +409,10 @@ __device__ __forceinline__ float half_row_max(const uint32_t (&s)[2][32], int kb
 // Returns the sum of the p.  Of every 8 pairs, EMU use the FMA-pipe exp2.
 // bf16 P (bf16 path) and f16 P (FP8 path) are rounded to nearest even; f16 P
 // (FP8 path) is rounded to nearest.
+// The second 32 values may still be in flight from TMEM: the loop waits for
+// them (a no-op when they have landed) before their chunk.
 template <class C, bool MASK, int EMU>
-__device__ __forceinline__ float half_row_exp_store(const uint32_t (&s)[2][32], uint32_t tS, int kbase, int valid,
+__device__ __forceinline__ float half_row_exp_store(uint32_t (&s)[2][32], uint32_t tS, int kbase, int valid,
                                                     float c2, float mc)
 {
     const float2 c2c2 = make_float2(c2, c2), nmc = make_float2(-mc, -mc);
@@ -418,6 +420,8 @@ __device__ __forceinline__ float half_row_exp_store(const uint32_t (&s)[2][32], 
                      make_float2(0.f, 0.f)};
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
+        if (i == 1)
+            tmem_wait_ld_regs(s[1]);
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
@@ -468,11 +472,14 @@ __device__ __forceinline__ void half_row_step(const PairCtx<C> &x, const FwdPara
         return;
     tc_fence_after();
     const uint32_t tS = x.tmem + lane_off + C::TM_S + 128u * buf + 64 * h;
+    // The first 32 values are waited for here; the second 32 load while the
+    // exponentials of the first run (the first tile needs all 64 for its max).
     uint32_t s[2][32];
     tmem_ld32(tS, s[0]);
-    tmem_ld32(tS + 32, s[1]);
     tmem_wait_ld_regs(s[0]);
-    tmem_wait_ld_regs(s[1]);
+    tmem_ld32(tS + 32, s[1]);
+    if (j == 0)
+        tmem_wait_ld_regs(s[1]);
     const bool masked = j == n - 1 && p.kv_tail < kBN;
     auto tile_max = [&]() {
         return masked ? half_row_max<true>(s, 64 * h, p.kv_tail) : half_row_max<false>(s, 64 * h, kBN);
@@ -491,9 +498,11 @@ __device__ __forceinline__ void half_row_step(const PairCtx<C> &x, const FwdPara
     if (j == 0)
         st.m_use = tile_max();
     sum = exp_store();
+    bool rescale = false;                    // warp-uniform: only the guard's path changes alpha
     if (j > 0) {
         const bool over = !(sum < (C::FP8 ? kPGuardF16 : kPGuardBF16));
         if (__any_sync(0xffffffffu, over)) {
+            rescale = true;
             if (over) {
                 const float mx = tile_max();
                 if (mx > st.m_use) {
@@ -505,7 +514,7 @@ __device__ __forceinline__ void half_row_step(const PairCtx<C> &x, const FwdPara
         }
     }
     st.l = st.l * alpha + sum;
-    if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+    if (rescale) {
         // Rescale this thread's row of O_h once PV(j-1) has finished with it.
         const int jp = j - 1;
         st.alive = __all_sync(0xffffffffu, wait_bar_cluster(x.bar(bars->pv_done[jp % 2]), (jp / 2) & 1,
