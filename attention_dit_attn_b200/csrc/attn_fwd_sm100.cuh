@@ -95,6 +95,7 @@ struct PCfg {
     static constexpr int THREADS = 384;
     static constexpr int REGS_SOFTMAX = 192, REGS_OTHER = 120;   // 2 x 192 + 120 = 3 x 168
     static constexpr int EXP_EMU = DIT_EXP_EMU;
+    static_assert(EXP_EMU >= 1 && 8 % EXP_EMU == 0, "polynomial pairs: 1, 2, 4 or 8 of every 8");
     static constexpr uint32_t IDESC_QK = FP8 ? make_idesc(kFmtE4M3, kFmtE4M3, 0, 2 * kBM, kBN)
                                              : make_idesc(kFmtBF16, kFmtBF16, 0, 2 * kBM, kBN);
     static constexpr uint32_t IDESC_PV = FP8 ? make_idesc(kFmtF16, kFmtF16, 1, 2 * kBM, D)
@@ -429,7 +430,11 @@ __device__ __forceinline__ float half_row_exp_store(uint32_t (&s)[2][32], uint32
             const float2 xv = __ffma2_rn(make_float2(__uint_as_float(s[i][c]), __uint_as_float(s[i][c + 1])),
                                          c2c2, nmc);
             float2 e;
-            if ((pi & 7) >= 8 - EMU) {
+            // Which EMU of every 8 pairs take the polynomial: the last ones on
+            // the bf16 path, every (8/EMU)-th one on the FP8 path (each measured
+            // faster on its own path).
+            const bool poly = C::FP8 ? (pi % (8 / EMU)) == (8 / EMU) - 1 : (pi & 7) >= 8 - EMU;
+            if (poly) {
                 e = exp2_poly2(xv);
             } else {
                 e.x = ex2_approx(xv.x);
