@@ -231,16 +231,16 @@ __device__ __forceinline__ void pair_producer(const PairCtx<C> &x, const FwdPara
 }
 
 // ------------------------------------------------------------------ MMA issuer (leader, one warp)
-// The whole warp runs the loop and one elected lane issues each MMA and
-// commit.  The issuing warp shares its SM sub-partition with two softmax
-// warps; in warp-uniform code the descriptor arithmetic stays on the uniform
-// datapath, which keeps the tensor pipe fed under that contention (a lone
-// lane-0 branch measured about 20% slower issue).  All shared-memory
-// descriptors of one operand differ only in the start-address field (bits
-// 0..13, address >> 4; addresses stay below 2^18 so the field never
-// carries), so each is a base descriptor plus a compile-time constant, and the
-// loop is unrolled over the two S buffers so that every TMEM address and
-// descriptor offset is an immediate.
+// The whole warp runs the loop and its waits; one elected lane issues all of a
+// step's MMAs and commits inside a single branch.  The issuing warp shares
+// its SM sub-partition with two softmax warps, and every instruction it
+// issues is taken from theirs: an election per MMA cost 1-4 % of the whole
+// kernel against one per step.  All shared-memory descriptors of one operand
+// differ only in the start-address field (bits 0..13, address >> 4;
+// addresses stay below 2^18 so the field never carries), so each is a base
+// descriptor plus a compile-time constant, and the loop is unrolled over the
+// two S buffers so that every TMEM address and descriptor offset is an
+// immediate.
 template <class C>
 __device__ __forceinline__ void pair_mma(const PairCtx<C> &x, const FwdParams &p)
 {
@@ -262,12 +262,10 @@ __device__ __forceinline__ void pair_mma(const PairCtx<C> &x, const FwdParams &p
             const uint32_t b = kk / C::STEPS_PER_BOX, w = (kk % C::STEPS_PER_BOX) * C::KSTEP;
             const uint64_t ad = q_desc + ((b * C::QBOX_BYTES + w) >> 4);
             const uint64_t bd = k_desc + ((BUF * K_STAGE + b * C::KBOX_BYTES + w) >> 4);
-            if (elect_one()) {
-                if (C::FP8)
-                    mma2_f8_ss(tmem + C::TM_S + 128u * BUF, ad, bd, C::IDESC_QK, kk > 0);
-                else
-                    mma2_f16_ss(tmem + C::TM_S + 128u * BUF, ad, bd, C::IDESC_QK, kk > 0);
-            }
+            if (C::FP8)
+                mma2_f8_ss(tmem + C::TM_S + 128u * BUF, ad, bd, C::IDESC_QK, kk > 0);
+            else
+                mma2_f16_ss(tmem + C::TM_S + 128u * BUF, ad, bd, C::IDESC_QK, kk > 0);
         }
     };
     // PV(j) from buffer BUF: key half h (P_h, V rows 64h..64h+63) into O_h.
@@ -277,9 +275,8 @@ __device__ __forceinline__ void pair_mma(const PairCtx<C> &x, const FwdParams &p
         for (int m = 0; m < 8; ++m) {
             const int h = m >> 2, kk = m & 3;
             const uint64_t bd = v_desc + ((BUF * V_STAGE + (64 * h + 16 * kk) * C::VROW) >> 4);
-            if (elect_one())
-                mma2_f16_ts(tmem + C::TM_O + h * C::D, tmem + C::TM_S + 128u * BUF + 64 * h + 8 * kk, bd,
-                            C::IDESC_PV, (kk == 0 && first) ? 0u : 1u);
+            mma2_f16_ts(tmem + C::TM_O + h * C::D, tmem + C::TM_S + 128u * BUF + 64 * h + 8 * kk, bd,
+                        C::IDESC_PV, (kk == 0 && first) ? 0u : 1u);
         }
     };
     bool ok = true;
@@ -294,13 +291,13 @@ __device__ __forceinline__ void pair_mma(const PairCtx<C> &x, const FwdParams &p
         if (!ok)
             return;
         tc_fence_after();
-        issue_pv(buf_c, j == 0);
-        if (elect_one())
+        if (elect_one()) {
+            issue_pv(buf_c, j == 0);
             mma2_commit_mc(x.bar(bars->pv_done[BUF]), kBoth);
-        if (j + 2 < n) {
-            issue_s(buf_c);
-            if (elect_one())
+            if (j + 2 < n) {
+                issue_s(buf_c);
                 mma2_commit_mc(x.bar(bars->s_full[BUF]), kBoth);
+            }
         }
         __syncwarp();
     };
@@ -310,13 +307,13 @@ __device__ __forceinline__ void pair_mma(const PairCtx<C> &x, const FwdParams &p
                                      wait_bar_cluster(x.bar(bars->k0_full), 0, x.abort, x.lim, kSiteKFull));
     if (ok) {
         tc_fence_after();
-        issue_s(B0{});
-        if (elect_one())
+        if (elect_one()) {
+            issue_s(B0{});
             mma2_commit_mc(x.bar(bars->s_full[0]), kBoth);
-        if (n > 1) {
-            issue_s(B1{});
-            if (elect_one())
+            if (n > 1) {
+                issue_s(B1{});
                 mma2_commit_mc(x.bar(bars->s_full[1]), kBoth);
+            }
         }
         __syncwarp();
     }
