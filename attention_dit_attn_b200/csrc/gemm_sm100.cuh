@@ -249,15 +249,18 @@ __device__ __forceinline__ void mma_issuer(const Ctx &x, const GemmParams &p)
             if (!ok)
                 break;
             tc_fence_after();
+            // One elected lane issues the stage's MMAs and its commit (one
+            // election per stage: fewer issue slots taken from the epilogue
+            // warps sharing this warp's sub-partition).
+            if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < Kind::MMAS_PER_STAGE; ++kk) {
-                const uint64_t ad = a_desc + ((uint32_t)(s * kStageA + kk * Kind::KSTEP_BYTES) >> 4);
-                const uint64_t bd = b_desc + ((uint32_t)(s * kStageB + kk * Kind::KSTEP_BYTES) >> 4);
-                if (elect_one())
+                for (int kk = 0; kk < Kind::MMAS_PER_STAGE; ++kk) {
+                    const uint64_t ad = a_desc + ((uint32_t)(s * kStageA + kk * Kind::KSTEP_BYTES) >> 4);
+                    const uint64_t bd = b_desc + ((uint32_t)(s * kStageB + kk * Kind::KSTEP_BYTES) >> 4);
                     mma2_f8_ss(acc, ad, bd, Kind::IDESC, (k > 0 || kk > 0) ? 1u : 0u);
-            }
-            if (elect_one())
+                }
                 mma2_commit_mc(x.bar(x.bars->empty[s]), kBoth);
+            }
             __syncwarp();
         }
         if (ok && elect_one())
@@ -689,17 +692,18 @@ __device__ __forceinline__ void p4_mma(const P4Ctx &x, const F4Params &p)
                 }
                 __syncwarp();
             }
+            // One elected lane issues the stage's MMAs and its commit.
+            if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const int g = kk >> 1;
-                const uint64_t ad = a_desc + ((uint32_t)(s * kP4StageA + kk * 32) >> 4);
-                const uint64_t bd = b_desc + ((uint32_t)(s * kP4StageB + kk * 32) >> 4);
-                if (elect_one())
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int g = kk >> 1;
+                    const uint64_t ad = a_desc + ((uint32_t)(s * kP4StageA + kk * 32) >> 4);
+                    const uint64_t bd = b_desc + ((uint32_t)(s * kP4StageB + kk * 32) >> 4);
                     mma2_mxf4(tmem, ad, bd, idesc_mxf4(2 * kF4BM, kF4BN, (uint32_t)(kk & 1) * 2u), sfa_t + 4 * g,
                               sfb_t + 8 * g, (k > 0 || kk > 0) ? 1u : 0u);
-            }
-            if (elect_one())
+                }
                 mma2_commit_mc(x.bar(x.bars->empty[s]), kBoth);
+            }
             __syncwarp();
         }
         if (ok && elect_one())
